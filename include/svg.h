@@ -1,0 +1,172 @@
+/*
+ * svg.h -- C ABI of the B200 semantic-aware top-p sparse attention library
+ * (libsvg.so, built for sm_100a).
+ *
+ * The five calls are the stages of the method described on the page
+ * "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
+ * Semantic-Aware Permutation" (technical summary, section 2):
+ *
+ *   svg_kmeans       section 2(a) "Clustering" + 2(c) "Centroid cache"
+ *   svg_permute      section 2(a) "Permutation"
+ *   svg_select_topp  section 2(b) "Centroid approximation" + "Top-p strategy"
+ *   svg_sparse_attn  section 2(c) "Customized attention kernel"
+ *   svg_unpermute    section 2(a) "Mathematical equivalence"
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are head-major: a [BH, N, D] tensor holds BH = batch*heads
+ *    independent heads of N tokens with D channels, row-major, contiguous.
+ *    Q/K/V and outputs are bfloat16 (raw 16-bit storage), centroids float32,
+ *    indices int32.  D must be 64 or 128.
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *    the pointer arrays `src`/`dst` of svg_permute, which are host arrays
+ *    holding device pointers.  The library never allocates or frees device
+ *    memory: scratch space comes from the caller as `ws`/`ws_bytes`, sized
+ *    with the matching *_workspace_size() call.  Workspaces need 256-byte
+ *    alignment and may be reused between calls on the same stream.
+ *  - Device pointers to bf16 tensors need 16-byte alignment.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Arguments are checked on the host before anything is
+ *    launched; a bad argument returns SVG_ERR_INVALID_ARG / _UNSUPPORTED /
+ *    _WORKSPACE and launches nothing.  A launch failure returns SVG_ERR_CUDA.
+ *  - Kernels never trap.  Every wait inside a kernel is bounded in time
+ *    (svg_set_wait_timeout_ns); when a bound is hit or a device-side check
+ *    fails the kernel records a code in a device error word and returns.
+ *    svg_get_error() reads and clears that word.
+ *  - Nothing throws across this boundary.
+ */
+#ifndef SVG_H_
+#define SVG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *svg_stream_t; /* same type as cudaStream_t */
+
+typedef enum svg_status {
+  SVG_OK = 0,
+  SVG_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, p out of range, C > N ... */
+  SVG_ERR_UNSUPPORTED = 2,  /* head dimension other than 64/128, sizes beyond int32 ranges */
+  SVG_ERR_WORKSPACE = 3,    /* ws smaller than the *_workspace_size() result */
+  SVG_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (launch, tensor map) */
+  SVG_ERR_TIMEOUT = 5,      /* a bounded in-kernel wait expired (device error word) */
+  SVG_ERR_DEVICE_CHECK = 6  /* a device-side consistency check failed (device error word) */
+} svg_status;
+
+/* Human-readable name of a status code (static string). */
+const char *svg_status_string(svg_status s);
+
+/* ------------------------------------------------------------------------ k-means
+ * Lloyd's k-means on every head independently (section 2(a) "Clustering":
+ * Q and K are clustered independently into C_q and C_k clusters).
+ *
+ *   x          [BH, N, D] bf16   tokens (Q or K of one layer)
+ *   centroids  [BH, C, D] fp32   in: initial centroids (seeding tokens, or the
+ *                                previous denoising step's centroids = the
+ *                                "centroid cache" of section 2(c));
+ *                                out: centroids after `iters` rounds
+ *   assign     [BH, N]    int32  out: cluster of every token, from the last
+ *                                assign step
+ *   counts     [BH, C]    int32  out: tokens per cluster for `assign`
+ *
+ * One round = assign (a_n = argmin_c ||x_n - mu_c||^2, ties to the lowest c)
+ * then update (mu_c = mean of its tokens, summed in fp64 in ascending token
+ * order; an empty cluster keeps its centroid).  The returned centroids are
+ * the means of the returned assignment.  Requires iters >= 1, 1 <= C <= N,
+ * C <= 1024.  Distances run on the tensor cores with the centroids split
+ * into a bf16 high and low part (about 16 significant bits).
+ */
+size_t svg_kmeans_workspace_size(int BH, int N, int D, int C);
+svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, float *centroids,
+                      int32_t *assign, int32_t *counts, void *ws, size_t ws_bytes,
+                      svg_stream_t stream);
+
+/* ------------------------------------------------------------------------ permutation
+ * Semantic-aware permutation (section 2(a) "Permutation"): a stable counting
+ * sort of the tokens of every head by cluster id, then a row gather.
+ *
+ *   assign   [BH, N]    int32  cluster ids in [0, C)
+ *   perm     [BH, N]    int32  out: perm[r] = source token of permuted row r;
+ *                              inside a cluster tokens keep ascending order
+ *   offsets  [BH, C+1]  int32  out: cluster c = rows [offsets[c], offsets[c+1])
+ *   src/dst  host arrays of `ntensors` (0..3) device pointers to [BH, N, D]
+ *            bf16 tensors; dst[t][h][r] = src[t][h][perm[h][r]].  Q uses the
+ *            Q permutation; K and V share the K permutation (call once with
+ *            ntensors = 2).  dst must not alias src.
+ * A device-side range check of `assign` records SVG_ERR_DEVICE_CHECK.
+ */
+size_t svg_permute_workspace_size(int BH, int N, int C);
+svg_status svg_permute(const int32_t *assign, int BH, int N, int C, int32_t *perm, int32_t *offsets,
+                       int ntensors, const void *const *src, void *const *dst, int D, void *ws,
+                       size_t ws_bytes, svg_stream_t stream);
+
+/* ------------------------------------------------------------------------ top-p selection
+ * Centroid-based top-p block selection (section 2(b)).  For every head h and
+ * q-cluster i with n_q[h,i] > 0:
+ *     logit_j = scale * mu_q[h,i] . mu_k[h,j]
+ *     w_j     = n_k[h,j] * exp(logit_j - max) / sum      (live j: n_k > 0)
+ * k-clusters are sorted by w descending (ties: lower j) and the shortest
+ * prefix whose cumulative weight reaches p is kept (p >= 1: every live j).
+ *
+ *   mu_q [BH, Cq, D] fp32, n_q [BH, Cq] int32, mu_k [BH, Ck, D] fp32, n_k [BH, Ck] int32
+ *   sel_count [BH, Cq]     int32  out: number of selected k-clusters (0 for empty rows)
+ *   sel_cols  [BH, Cq, Ck] int32  out: row (h,i) holds its selected k-cluster ids in
+ *                                 ascending order in its first sel_count entries;
+ *                                 the remaining entries are left untouched
+ * Requires 0 < p, Ck <= 1024; scale <= 0 selects 1/sqrt(D).  All math fp32.
+ */
+svg_status svg_select_topp(const float *mu_q, const int32_t *n_q, const float *mu_k,
+                           const int32_t *n_k, int BH, int Cq, int Ck, int D, float p, float scale,
+                           int32_t *sel_count, int32_t *sel_cols, svg_stream_t stream);
+
+/* ------------------------------------------------------------------------ sparse attention
+ * Attention over the selected variable-size blocks (section 2(c) "Customized
+ * attention kernel"): permuted query rows of q-cluster i attend, with exact
+ * softmax and no causal mask, to the union of the permuted key rows of the
+ * k-clusters selected for i.
+ *
+ *   qp, kp, vp  [BH, N, D] bf16  permuted Q (Q permutation), K and V (K permutation)
+ *   q_off       [BH, Cq+1] int32 q-cluster row ranges (svg_permute offsets)
+ *   k_off       [BH, Ck+1] int32 k-cluster row ranges
+ *   sel_count, sel_cols          svg_select_topp output
+ *   op          [BH, N, D] bf16  out: permuted output rows
+ *   lse         [BH, N]    fp32  optional out (NULL to skip): natural-log
+ *                                sum_j exp(scale * q.k_j) per row
+ * Rows of empty q-clusters do not exist; every other row is written.  A row
+ * whose cluster selected no key is left untouched and flagged with
+ * SVG_ERR_DEVICE_CHECK.  scale <= 0 selects 1/sqrt(D).
+ */
+size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq);
+svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
+                           const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
+                           const int32_t *sel_count, const int32_t *sel_cols, float scale, void *op,
+                           float *lse, void *ws, size_t ws_bytes, svg_stream_t stream);
+
+/* ------------------------------------------------------------------------ un-permutation
+ * Inverse permutation (section 2(a) "Mathematical equivalence"):
+ * x[h][perm[h][r]] = xp[h][r] for every row r.  x must not alias xp.
+ */
+svg_status svg_unpermute(const void *xp, const int32_t *perm, int BH, int N, int D, void *x,
+                         svg_stream_t stream);
+
+/* ------------------------------------------------------------------------ errors and limits
+ * svg_get_error synchronises `stream`, then returns and clears the device
+ * error word of the current device (SVG_OK when nothing was recorded;
+ * SVG_ERR_CUDA when the synchronisation itself failed).
+ * svg_set_wait_timeout_ns sets the bound of every in-kernel wait for the
+ * following launches (default 2e9 ns; 0 restores the default).
+ */
+svg_status svg_get_error(svg_stream_t stream);
+void svg_set_wait_timeout_ns(uint64_t ns);
+
+/* Library version, e.g. "svg-b200 0.1 (sm_100a)". */
+const char *svg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVG_H_ */

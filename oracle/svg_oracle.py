@@ -175,10 +175,14 @@ class RowSelection:
     undecided: bool           # the cut sits within `tol` of a float32-visible boundary
 
 
-def select_row(weights: np.ndarray, p: float, tol: float = 1e-4) -> RowSelection:
-    """Smallest prefix of the descending-score order whose mass reaches p."""
+def select_row(weights: np.ndarray, p: float, tol: float = 1e-4,
+               live_mask: Optional[np.ndarray] = None) -> RowSelection:
+    """Smallest prefix of the descending-score order whose mass reaches p.
+
+    ``live_mask`` marks the non-empty k-clusters (default: weight > 0).
+    """
     w = np.asarray(weights, np.float64)
-    live = np.nonzero(w > 0)[0]
+    live = np.nonzero(w > 0 if live_mask is None else np.asarray(live_mask))[0]
     if len(live) == 0:
         return RowSelection(np.zeros(0, np.int64), live, w, False)
     # descending weight, ties -> lower index (stable sort of ascending index list)
@@ -204,7 +208,8 @@ def select_topp(mu_q: np.ndarray, n_q: np.ndarray, mu_k: np.ndarray, n_k: np.nda
             rows.append(RowSelection(np.zeros(0, np.int64), np.zeros(0, np.int64),
                                      np.zeros(mu_k.shape[0]), False))
             continue
-        rows.append(select_row(centroid_weights(mu_q[i], mu_k, n_k, scale), p, tol))
+        rows.append(select_row(centroid_weights(mu_q[i], mu_k, n_k, scale), p, tol,
+                               np.asarray(n_k) > 0))
     return rows
 
 

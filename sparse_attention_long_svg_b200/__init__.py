@@ -1,0 +1,302 @@
+"""Python binding of libsvg.so (semantic-aware top-p sparse attention, B200).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+of libsvg.so, reached through its C ABI (include/svg.h) with ctypes.
+PyTorch supplies device memory and the current CUDA stream.  There is no
+CPU fallback: importing works without a GPU, but every call needs the built
+library and a CUDA device and raises otherwise.
+
+Stages (Sparse VideoGen2, section 2): ``kmeans`` -> ``permute`` ->
+``select_topp`` -> ``sparse_attn`` -> ``unpermute``; ``svg_attention`` runs
+the whole layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvg.so")
+
+STATUS = {0: "SVG_OK", 1: "SVG_ERR_INVALID_ARG", 2: "SVG_ERR_UNSUPPORTED", 3: "SVG_ERR_WORKSPACE",
+          4: "SVG_ERR_CUDA", 5: "SVG_ERR_TIMEOUT", 6: "SVG_ERR_DEVICE_CHECK"}
+
+# name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "svg_status_string": (ctypes.c_char_p, [_I]),
+    "svg_version": (ctypes.c_char_p, []),
+    "svg_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
+    "svg_get_error": (_I, [_P]),
+    "svg_kmeans_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "svg_kmeans": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "svg_permute_workspace_size": (_SZ, [_I, _I, _I]),
+    "svg_permute": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _SZ, _P]),
+    "svg_select_topp": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P, _P, _P]),
+    "svg_sparse_attn_workspace_size": (_SZ, [_I, _I, _I]),
+    "svg_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _SZ, _P]),
+    "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+}
+
+_lib = None
+
+
+class SvgError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsvg.so (no CUDA device needed) and declares every ABI symbol."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m sparse_attention_long_svg_b200.build` "
+                           "(or __graft_entry__.build()); there is no CPU fallback")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(name: str, status: int):
+    if status != 0:
+        raise SvgError(name, status)
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, dims: int):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def get_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word."""
+    return load_library().svg_get_error(_stream(stream))
+
+
+def set_wait_timeout_ns(ns: int):
+    load_library().svg_set_wait_timeout_ns(int(ns))
+
+
+# --------------------------------------------------------------------- stages
+
+def kmeans(x: torch.Tensor, centroids: torch.Tensor, iters: int, assign: Optional[torch.Tensor] = None,
+           counts: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """k-means of every head of x [BH, N, D] bf16, updating centroids [BH, C, D] fp32 in place.
+
+    Returns (centroids, assign [BH, N] int32, counts [BH, C] int32).
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16, 3)
+    _need(centroids, "centroids", torch.float32, 3)
+    BH, N, D = x.shape
+    C = centroids.shape[1]
+    if assign is None:
+        assign = torch.empty((BH, N), dtype=torch.int32, device=x.device)
+    if counts is None:
+        counts = torch.empty((BH, C), dtype=torch.int32, device=x.device)
+    nbytes = lib.svg_kmeans_workspace_size(BH, N, D, C)
+    if workspace is None:
+        workspace = _ws(nbytes, x.device)
+    _check("svg_kmeans", lib.svg_kmeans(_ptr(x), BH, N, D, C, int(iters), _ptr(centroids), _ptr(assign),
+                                        _ptr(counts), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return centroids, assign, counts
+
+
+def permute(assign: torch.Tensor, C: int, tensors: Sequence[torch.Tensor] = (),
+            out: Optional[Sequence[torch.Tensor]] = None, perm: Optional[torch.Tensor] = None,
+            offsets: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Stable counting sort by cluster and row gather of up to 3 [BH, N, D] bf16 tensors.
+
+    Returns (perm [BH, N] int32, offsets [BH, C+1] int32, permuted tensors).
+    """
+    lib = load_library()
+    _need(assign, "assign", torch.int32, 2)
+    BH, N = assign.shape
+    dev = assign.device
+    tensors = list(tensors)
+    if out is None:
+        out = [torch.empty_like(t) for t in tensors]
+    out = list(out)
+    D = tensors[0].shape[2] if tensors else 64
+    for t in tensors + out:
+        _need(t, "tensor", torch.bfloat16, 3)
+    if perm is None:
+        perm = torch.empty((BH, N), dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty((BH, C + 1), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = _ws(lib.svg_permute_workspace_size(BH, N, C), dev)
+    n = len(tensors)
+    src = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in tensors])
+    dst = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in out])
+    _check("svg_permute", lib.svg_permute(_ptr(assign), BH, N, int(C), _ptr(perm), _ptr(offsets), n,
+                                          ctypes.cast(src, ctypes.c_void_p), ctypes.cast(dst, ctypes.c_void_p),
+                                          int(D), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return perm, offsets, out
+
+
+def select_topp(mu_q: torch.Tensor, n_q: torch.Tensor, mu_k: torch.Tensor, n_k: torch.Tensor, p: float,
+                scale: float = 0.0, sel_count: Optional[torch.Tensor] = None,
+                sel_cols: Optional[torch.Tensor] = None, stream=None):
+    """Top-p (q-cluster, k-cluster) block selection.  Returns (sel_count [BH, Cq], sel_cols [BH, Cq, Ck])."""
+    lib = load_library()
+    _need(mu_q, "mu_q", torch.float32, 3)
+    _need(mu_k, "mu_k", torch.float32, 3)
+    _need(n_q, "n_q", torch.int32, 2)
+    _need(n_k, "n_k", torch.int32, 2)
+    BH, Cq, D = mu_q.shape
+    Ck = mu_k.shape[1]
+    if sel_count is None:
+        sel_count = torch.empty((BH, Cq), dtype=torch.int32, device=mu_q.device)
+    if sel_cols is None:
+        sel_cols = torch.empty((BH, Cq, Ck), dtype=torch.int32, device=mu_q.device)
+    _check("svg_select_topp", lib.svg_select_topp(_ptr(mu_q), _ptr(n_q), _ptr(mu_k), _ptr(n_k), BH, Cq, Ck, D,
+                                                  float(p), float(scale), _ptr(sel_count), _ptr(sel_cols),
+                                                  _stream(stream)))
+    return sel_count, sel_cols
+
+
+def sparse_attn(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
+                want_lse: bool = False, lse=None, workspace=None, stream=None):
+    """Attention over the selected blocks of permuted Q/K/V.  Returns (op, lse or None)."""
+    lib = load_library()
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
+        _need(t, n, torch.bfloat16, 3)
+    BH, N, D = qp.shape
+    Cq = q_off.shape[1] - 1
+    Ck = k_off.shape[1] - 1
+    if op is None:
+        op = torch.empty_like(qp)
+    if want_lse and lse is None:
+        lse = torch.empty((BH, N), dtype=torch.float32, device=qp.device)
+    if workspace is None:
+        workspace = _ws(lib.svg_sparse_attn_workspace_size(BH, N, Cq), qp.device)
+    _check("svg_sparse_attn", lib.svg_sparse_attn(
+        _ptr(qp), _ptr(kp), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
+        _ptr(sel_cols), float(scale), _ptr(op), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return op, lse
+
+
+def unpermute(xp: torch.Tensor, perm: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """x[h, perm[h, r]] = xp[h, r]."""
+    lib = load_library()
+    _need(xp, "xp", torch.bfloat16, 3)
+    BH, N, D = xp.shape
+    if out is None:
+        out = torch.empty_like(xp)
+    _check("svg_unpermute", lib.svg_unpermute(_ptr(xp), _ptr(perm), BH, N, D, _ptr(out), _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------- the layer
+
+@dataclass
+class LayerState:
+    """Everything one layer call produces; centroids are the next call's warm start."""
+    mu_q: torch.Tensor
+    mu_k: torch.Tensor
+    assign_q: torch.Tensor
+    assign_k: torch.Tensor
+    n_q: torch.Tensor
+    n_k: torch.Tensor
+    perm_q: torch.Tensor
+    perm_k: torch.Tensor
+    q_off: torch.Tensor
+    k_off: torch.Tensor
+    sel_count: torch.Tensor
+    sel_cols: torch.Tensor
+    qp: torch.Tensor
+    kp: torch.Tensor
+    vp: torch.Tensor
+    op: torch.Tensor
+
+
+class SvgLayer:
+    """Preallocated buffers for repeated layer calls of one shape (no allocation per call)."""
+
+    def __init__(self, BH: int, N: int, D: int, Cq: int, Ck: int, device="cuda"):
+        lib = load_library()
+        self.shape = (BH, N, D, Cq, Ck)
+        i32 = dict(dtype=torch.int32, device=device)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.assign_q = torch.empty((BH, N), **i32)
+        self.assign_k = torch.empty((BH, N), **i32)
+        self.n_q = torch.empty((BH, Cq), **i32)
+        self.n_k = torch.empty((BH, Ck), **i32)
+        self.perm_q = torch.empty((BH, N), **i32)
+        self.perm_k = torch.empty((BH, N), **i32)
+        self.q_off = torch.empty((BH, Cq + 1), **i32)
+        self.k_off = torch.empty((BH, Ck + 1), **i32)
+        self.sel_count = torch.empty((BH, Cq), **i32)
+        self.sel_cols = torch.empty((BH, Cq, Ck), **i32)
+        self.qp = torch.empty((BH, N, D), **bf)
+        self.kp = torch.empty((BH, N, D), **bf)
+        self.vp = torch.empty((BH, N, D), **bf)
+        self.op = torch.empty((BH, N, D), **bf)
+        ws = max(lib.svg_kmeans_workspace_size(BH, N, D, Cq), lib.svg_kmeans_workspace_size(BH, N, D, Ck),
+                 lib.svg_permute_workspace_size(BH, N, max(Cq, Ck)),
+                 lib.svg_sparse_attn_workspace_size(BH, N, Cq))
+        self.workspace = _ws(ws, device)
+
+    def __call__(self, q, k, v, mu_q, mu_k, iters: int, p: float, scale: float = 0.0, out=None, stream=None):
+        kmeans(q, mu_q, iters, self.assign_q, self.n_q, self.workspace, stream)
+        kmeans(k, mu_k, iters, self.assign_k, self.n_k, self.workspace, stream)
+        Cq, Ck = mu_q.shape[1], mu_k.shape[1]
+        permute(self.assign_q, Cq, [q], [self.qp], self.perm_q, self.q_off, self.workspace, stream)
+        permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace, stream)
+        select_topp(mu_q, self.n_q, mu_k, self.n_k, p, scale, self.sel_count, self.sel_cols, stream)
+        sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,
+                    self.op, workspace=self.workspace, stream=stream)
+        out = unpermute(self.op, self.perm_q, out, stream)
+        return out, LayerState(mu_q, mu_k, self.assign_q, self.assign_k, self.n_q, self.n_k, self.perm_q,
+                               self.perm_k, self.q_off, self.k_off, self.sel_count, self.sel_cols, self.qp,
+                               self.kp, self.vp, self.op)
+
+
+def svg_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mu_q: torch.Tensor, mu_k: torch.Tensor,
+                  iters: int, p: float, scale: float = 0.0):
+    """One SVG2 attention layer: returns (out [BH, N, D] bf16, LayerState).
+
+    mu_q / mu_k [BH, C, D] fp32 hold the initial centroids (seeding tokens or
+    the previous step's cache) and are updated in place.
+    """
+    BH, N, D = q.shape
+    layer = SvgLayer(BH, N, D, mu_q.shape[1], mu_k.shape[1], q.device)
+    return layer(q, k, v, mu_q, mu_k, iters, p, scale)
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

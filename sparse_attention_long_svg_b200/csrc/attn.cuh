@@ -1,0 +1,621 @@
+// Varlen block-sparse attention over the selected (q-cluster, k-cluster)
+// blocks (Sparse VideoGen2, section 2(c) "Customized attention kernel": the
+// query rows of a cluster are contiguous after the permutation and are
+// computed densely; the selected key clusters are scattered ranges of the
+// permuted K/V and are gathered sparsely, without padding them to fixed
+// block sizes).
+//
+// Work unit: 128 consecutive permuted query rows of one q-cluster ("q-tile").
+// Its key list is the concatenation of the selected k-clusters' row ranges,
+// cut into 8-row slots; 16 slots form a 128-key tile.  A k-cluster of n rows
+// costs ceil(n/8) slots and at most 7 masked rows; it is fetched with as few
+// TMA boxes as possible (boxes of 8..128 rows, a power of two that fits the
+// rest of the cluster and the rest of the tile).  Rows past a cluster's end
+// inside its last slot are masked out of the softmax.
+//
+// Per CTA (persistent, one per SM), 7 warps:
+//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t)
+//   warp 4     TMA producer: Q tile, K and V boxes into 2- and 3-stage rings
+//   warp 5     MMA issuer: S = Q K^T into TMEM (double-buffered) and
+//              O += P V into TMEM; issues whichever of the two is ready
+//              first; also owns the TMEM allocation
+//   warp 6     item loader: the next q-tile's selected key ranges, read from
+//              global memory into a 2-entry shared-memory ring ahead of time
+// Per key tile k: S(k) -> softmax(k) writes P(k) (bf16 pairs, TMEM) ->
+// PV(k) with A = P read from TMEM.  O accumulates in TMEM across the key tiles of a q-tile; the softmax
+// warps rescale it in place only when a row's running max grows by more than
+// 2^8 (exact: every probability is taken against the same reference max that
+// O and the row sum use).
+#pragma once
+#include "common.cuh"
+
+namespace svg {
+
+struct AttnItem {  // one q-tile
+  int32_t h, i, q0, packed;  // packed = rows (<=128) | key_tiles << 8
+};
+
+template <int D>
+struct AttnCfg {
+  static constexpr int BM = 128, BN = 128, SLOT = 8, NSLOT = BN / SLOT;
+  static constexpr int DH = D / 64;  // 64-channel (128-byte) halves
+  static constexpr int KST = 2;      // K ring depth
+  static constexpr int VST = 3;      // V ring depth (V(t) is issued only once PV(t - VST) is done)
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int HALF_Q = BM * 128;   // bytes of one 64-channel half of Q
+  static constexpr int HALF_KV = BN * 128;  // same for a K/V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int MAX_SEL = 1024;                      // selected k-clusters per q-cluster
+  static constexpr int OFF_RANGES = OFF_V + VST * KV_BYTES; // 2 x int2 (first row, rows) per selection
+  static constexpr int OFF_BAR = OFF_RANGES + 2 * MAX_SEL * 8;
+  static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers/meta + alignment slack
+  static constexpr uint32_t TM_S = 0;      // two S buffers: columns [0,128) and [128,256)
+  static constexpr uint32_t TM_O = 256;    // O: columns [256, 256 + D)
+  static constexpr uint32_t TM_P = 384;    // P (bf16 pairs): columns [384, 448)
+  static constexpr uint32_t TM_COLS = 512;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+  static constexpr int THREADS = 224;
+};
+
+// TMA boxes of 8, 16, 32, 64 and 128 rows (one tensor map each for K and V).
+constexpr int kNumBoxSizes = 5;
+
+struct AttnMaps {
+  CUtensorMap q;
+  CUtensorMap k[kNumBoxSizes];
+  CUtensorMap v[kNumBoxSizes];
+};
+
+// Sets bits [first, first + count) of a 128-bit mask held in four registers
+// (word-level arithmetic; no per-bit loop, no dynamic indexing).
+__device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count) {
+  const int last = first + count;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int lo = max(first, 32 * w), hi = min(last, 32 * w + 32);
+    if (hi > lo) {
+      const int n = hi - lo;
+      const uint32_t bits = n >= 32 ? 0xFFFFFFFFu : ((1u << n) - 1u);
+      m[w] |= bits << (lo - 32 * w);
+    }
+  }
+}
+
+struct AttnBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[2], k_empty[2], v_full[3], v_empty[3], meta_full[3];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, o_full;
+  uint64_t item_full[2], item_empty[2];
+  uint64_t drain;
+  AttnItem item[2];      // item ring written by the loader warp
+  int32_t item_cnt[2];
+  uint32_t meta[3][4];   // per V stage: 128-bit key validity mask of the tile
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+struct AttnParams {
+  const int32_t *q_off, *k_off, *sel_count, *sel_cols;
+  const AttnItem *items;
+  const int32_t *num_items;
+  __nv_bfloat16 *op;
+  float *lse;
+  int N, Cq, Ck, BH;
+  float scale_log2;      // softmax scale * log2(e)
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ bool attn_wait(AttnBarriers *b, uint64_t *bar, uint32_t parity,
+                                          uint64_t ns, uint32_t site) {
+  if (mbar_wait(bar, parity, ns)) return true;
+  record_error(SVG_ERR_TIMEOUT, site);
+  atomicExch(&b->abort_flag, 1);
+  return false;
+}
+
+__device__ __forceinline__ bool aborted(AttnBarriers *b) {
+  return *reinterpret_cast<volatile int32_t *>(&b->abort_flag) != 0;
+}
+
+// Every lane waits; the warp proceeds only if all lanes saw the phase, so the
+// .sync.aligned tcgen05 loads that follow always run on the full warp.
+__device__ __forceinline__ bool attn_warp_wait(AttnBarriers *b, uint64_t *bar, uint32_t parity,
+                                               uint64_t ns, uint32_t site) {
+  const bool ok = mbar_wait(bar, parity, ns);
+  const bool all = __all_sync(0xffffffffu, ok);
+  if (!all && lane_id() == 0) {
+    record_error(SVG_ERR_TIMEOUT, site);
+    atomicExch(&b->abort_flag, 1);
+  }
+  return all;
+}
+
+__device__ __forceinline__ bool warp_aborted(AttnBarriers *b) {
+  return __any_sync(0xffffffffu, aborted(b));
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
+    sparse_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams P) {
+  using Cfg = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem + Cfg::OFF_Q;
+  uint8_t *sK = smem + Cfg::OFF_K;
+  uint8_t *sV = smem + Cfg::OFF_V;
+  int2 *sRanges = reinterpret_cast<int2 *>(smem + Cfg::OFF_RANGES);
+  AttnBarriers *B = reinterpret_cast<AttnBarriers *>(smem + Cfg::OFF_BAR);
+  const int warp = static_cast<int>(warp_id());
+  const int lane = static_cast<int>(lane_id());
+
+  if (threadIdx.x == 0) {
+    mbar_init(&B->q_full, 1);
+    mbar_init(&B->q_empty, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&B->v_full[s], 1);
+      mbar_init(&B->v_empty[s], 1);
+      mbar_init(&B->meta_full[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&B->k_full[s], 1);
+      mbar_init(&B->k_empty[s], 1);
+      mbar_init(&B->s_full[s], 1);
+      mbar_init(&B->s_free[s], 4);
+      mbar_init(&B->item_full[s], 1);
+      mbar_init(&B->item_empty[s], 1);
+    }
+    mbar_init(&B->p_full, 4);
+    mbar_init(&B->o_full, 1);
+    mbar_init(&B->drain, 1);
+    B->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&B->tmem_base, Cfg::TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&maps.q);
+    for (int b = 0; b < kNumBoxSizes; ++b) {
+      tma_prefetch_desc(&maps.k[b]);
+      tma_prefetch_desc(&maps.v[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B->tmem_base;
+  const int total = *P.num_items;
+  const uint64_t ns = P.wait_ns;
+  const int grid = static_cast<int>(gridDim.x);
+
+  if (warp == 6) {
+    // ------------------------------------------------------------ item loader
+    int n = 0;
+    for (int w = blockIdx.x; w < total; w += grid, ++n) {
+      const int buf = n & 1;
+      bool ok = true;
+      if (lane == 0 && n >= 2)
+        ok = attn_wait(B, &B->item_empty[buf], ((n >> 1) - 1) & 1, ns, SITE_ATTN_PRODUCER);
+      if (!__shfl_sync(0xffffffffu, ok, 0) || warp_aborted(B)) break;
+      const AttnItem it = P.items[w];
+      const int cnt = min(P.sel_count[it.h * P.Cq + it.i], Cfg::MAX_SEL);
+      const int32_t *cols = P.sel_cols + static_cast<size_t>(it.h * P.Cq + it.i) * P.Ck;
+      const int32_t *koff = P.k_off + static_cast<size_t>(it.h) * (P.Ck + 1);
+      int2 *dst = sRanges + buf * Cfg::MAX_SEL;
+      for (int c = lane; c < cnt; c += 32) {
+        const int j = cols[c];
+        int2 r = make_int2(0, 0);  // out-of-range ids are flagged by the planning kernel
+        if (j >= 0 && j < P.Ck) {
+          r.x = koff[j];
+          r.y = koff[j + 1] - r.x;
+        }
+        dst[c] = r;
+      }
+      if (lane == 0) {
+        B->item[buf] = it;
+        B->item_cnt[buf] = cnt;
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B->item_full[buf]);
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    uint32_t g = 0;  // global key-tile counter
+    int n_items = 0;
+    if (lane == 0) {
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok && !aborted(B); w += grid, ++n_items) {
+        const int buf = n_items & 1;
+        if (!attn_wait(B, &B->item_full[buf], (n_items >> 1) & 1, ns, SITE_ATTN_PRODUCER)) break;
+        const AttnItem it = B->item[buf];
+        const int cnt = B->item_cnt[buf];
+        const int2 *ranges = sRanges + buf * Cfg::MAX_SEL;
+        const int ntk = it.packed >> 8;
+        if (n_items > 0 && !attn_wait(B, &B->q_empty, (n_items - 1) & 1, ns, SITE_ATTN_PRODUCER))
+          break;
+        mbar_arrive_expect_tx(&B->q_full, Cfg::Q_BYTES);
+        const int qrow = it.h * P.N + it.q0;
+#pragma unroll
+        for (int dh = 0; dh < Cfg::DH; ++dh)
+          tma_load_2d(sQ + dh * Cfg::HALF_Q, &maps.q, dh * 64, qrow, &B->q_full);
+        int ci = 0, cur = 0, left = 0;
+        const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
+        for (int t = 0; t < ntk; ++t, ++g) {
+          const int st = g & 1;
+          const uint32_t ph = (g >> 1) & 1;
+          const int vs = static_cast<int>(g % 3);
+          const uint32_t vph = (g / 3) & 1;
+          // Cut the tile into boxes of 1, 2, 4, 8 or 16 slots (8..128 rows): the
+          // largest power of two that fits both the tile and the cluster rest.
+          int box_row[Cfg::NSLOT], box_kind[Cfg::NSLOT], nbox = 0;
+          uint32_t mask[4] = {0, 0, 0, 0};
+          int sl = 0;
+          while (sl < Cfg::NSLOT) {
+            while (left <= 0 && ci < cnt) {
+              const int2 r = ranges[ci++];
+              cur = r.x;
+              left = r.y;
+            }
+            const int space = Cfg::NSLOT - sl;
+            const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
+            int kind = 0;
+            while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
+            const int nsl = 1 << kind;
+            if (left > 0) {
+              set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
+              box_row[nbox] = it.h * P.N + cur;
+              cur += nsl * Cfg::SLOT;
+              left -= nsl * Cfg::SLOT;
+            } else {
+              box_row[nbox] = pad_row;   // no keys left: finite filler rows, masked out
+            }
+            box_kind[nbox] = kind | (sl << 8);
+            ++nbox;
+            sl += nsl;
+          }
+          if (g >= 2 && !attn_wait(B, &B->k_empty[st], ph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(&B->k_full[st], Cfg::KV_BYTES);
+          uint8_t *kdst = sK + st * Cfg::KV_BYTES;
+          for (int bx = 0; bx < nbox; ++bx) {
+            const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
+#pragma unroll
+            for (int dh = 0; dh < Cfg::DH; ++dh)
+              tma_load_2d(kdst + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64, box_row[bx],
+                          &B->k_full[st]);
+          }
+          if (g >= 3 && !attn_wait(B, &B->v_empty[vs], vph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
+          B->meta[vs][0] = mask[0];
+          B->meta[vs][1] = mask[1];
+          B->meta[vs][2] = mask[2];
+          B->meta[vs][3] = mask[3];
+          mbar_arrive(&B->meta_full[vs]);
+          mbar_arrive_expect_tx(&B->v_full[vs], Cfg::KV_BYTES);
+          uint8_t *vdst = sV + vs * Cfg::KV_BYTES;
+          for (int bx = 0; bx < nbox; ++bx) {
+            const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
+#pragma unroll
+            for (int dh = 0; dh < Cfg::DH; ++dh)
+              tma_load_2d(vdst + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64, box_row[bx],
+                          &B->v_full[vs]);
+          }
+        }
+        mbar_arrive(&B->item_empty[buf]);   // the ranges of this item are no longer read
+      }
+      // drain: every load issued above lands on a full barrier; wait for the
+      // last phase of each so no copy is in flight when the CTA exits.
+      if (aborted(B)) {
+        if (n_items > 0) mbar_wait(&B->q_full, (n_items - 1) & 1, 1000000000ull);
+        for (uint32_t k = (g >= 3 ? g - 3 : 0); k < g; ++k) {
+          mbar_wait(&B->k_full[k & 1], (k >> 1) & 1, 1000000000ull);
+          mbar_wait(&B->v_full[k % 3], (k / 3) & 1, 1000000000ull);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    // Two cursors walk this CTA's key tiles: gs = next S, gp = next PV.  Each
+    // pass issues whichever is ready (S first), so neither waits behind the
+    // other's operands.  S may run at most two tiles ahead (two S buffers).
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      int ws = blockIdx.x, wp = blockIdx.x, n_s = 0;
+      int ts = 0, tp = 0;
+      int ntk_s = ws < total ? (P.items[ws].packed >> 8) : 0;
+      int ntk_p = ntk_s;
+      int ntk_next = ws + grid < total ? (P.items[ws + grid].packed >> 8) : 0;
+      uint32_t gs = 0, gp = 0;
+      bool q_ok = false;
+      const long long limit = static_cast<long long>(ns) * 2;
+      long long t_last = clock64();
+      while (wp < total) {
+        bool progress = false;
+        if (ws < total && gs < gp + 2) {
+          if (!q_ok) q_ok = mbar_try_wait(&B->q_full, n_s & 1);
+          const int st = gs & 1;
+          if (q_ok && mbar_try_wait(&B->k_full[st], (gs >> 1) & 1) &&
+              (gs < 2 || mbar_try_wait(&B->s_free[st], ((gs >> 1) - 1) & 1))) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * Cfg::HALF_Q + (kk & 3) * 32;
+              const uint64_t a = smem_desc_sw128(q_base + koff, 16, 1024);
+              const uint64_t b = smem_desc_sw128(
+                  k_base + st * Cfg::KV_BYTES + (kk >> 2) * Cfg::HALF_KV + (kk & 3) * 32, 16, 1024);
+              mma_bf16_ss(tmem + Cfg::TM_S + st * 128, a, b, Cfg::IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&B->s_full[st]);
+            mma_commit(&B->k_empty[st]);
+            if (++ts == ntk_s) {            // last S of this item: Q may be replaced
+              mma_commit(&B->q_empty);
+              ws += grid;
+              ++n_s;
+              ts = 0;
+              ntk_s = ntk_next;
+              ntk_next = ws + grid < total ? (P.items[ws + grid].packed >> 8) : 0;
+              q_ok = false;
+            }
+            ++gs;
+            progress = true;
+          }
+        }
+        if (gp < gs) {
+          const int vs = static_cast<int>(gp % 3);
+          if (mbar_try_wait(&B->p_full, gp & 1) && mbar_try_wait(&B->v_full[vs], (gp / 3) & 1)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < Cfg::BN / 16; ++kk) {
+              // A = P [128 q x 16 keys] in TMEM; B = V [16 keys x D] in smem, MN-major
+              const uint64_t b = smem_desc_sw128(v_base + vs * Cfg::KV_BYTES + kk * 2048,
+                                                 Cfg::HALF_KV, 1024);
+              mma_bf16_ts(tmem + Cfg::TM_O, tmem + Cfg::TM_P + kk * 8, b, Cfg::IDESC_PV,
+                          (tp == 0 && kk == 0) ? 0u : 1u);
+            }
+            mma_commit(&B->o_full);
+            mma_commit(&B->v_empty[vs]);
+            if (++tp == ntk_p) {
+              wp += grid;
+              tp = 0;
+              ntk_p = wp < total ? (P.items[wp].packed >> 8) : 0;
+            }
+            ++gp;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (clock64() - t_last > limit) {
+          record_error(SVG_ERR_TIMEOUT, SITE_ATTN_MMA);
+          atomicExch(&B->abort_flag, 1);
+          break;
+        } else if (aborted(B)) {
+          break;
+        }
+      }
+      // make sure every issued MMA has retired before TMEM is released
+      mma_commit(&B->drain);
+      mbar_wait(&B->drain, 0, 1000000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    // Thread `row` owns TMEM lane `row`: one query row of S and of O.
+    // Probabilities are taken against a reference max m_ref that is raised
+    // only when a tile's max exceeds it by more than kRescaleLog2; O (in
+    // TMEM) and l are rescaled then.  P values stay below 2^kRescaleLog2.
+    constexpr float kRescaleLog2 = 8.f;
+    const int row = threadIdx.x;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t o_addr = tmem + lane_off + Cfg::TM_O;
+    const float sl2 = P.scale_log2;
+    uint32_t g = 0, s_iter = 0, pv_iter = 0;
+    AttnItem next_it = blockIdx.x < total ? P.items[blockIdx.x] : AttnItem{0, 0, 0, 0};
+    for (int w = blockIdx.x; w < total && !warp_aborted(B); w += gridDim.x) {
+      const AttnItem it = next_it;
+      if (w + static_cast<int>(gridDim.x) < total) next_it = P.items[w + gridDim.x];  // prefetch
+      const int ntk = it.packed >> 8;
+      const int nrows = it.packed & 0xFF;
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int t = 0; t < ntk; ++t, ++g, ++s_iter) {
+        const int st = static_cast<int>(g % 3);
+        const uint32_t ph = (g / 3) & 1;
+        const uint32_t sb = s_iter & 1;
+        if (!attn_warp_wait(B, &B->s_full[sb], (s_iter >> 1) & 1, ns, SITE_ATTN_SOFTMAX) ||
+            !attn_warp_wait(B, &B->meta_full[st], ph, ns, SITE_ATTN_SOFTMAX)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t mk[4] = {B->meta[st][0], B->meta[st][1], B->meta[st][2], B->meta[st][3]};
+        const uint32_t s_addr = tmem + lane_off + Cfg::TM_S + sb * 128;
+        float sv[4][32];
+        tmem_ld128_sync(s_addr, reinterpret_cast<float(&)[128]>(sv));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->s_free[sb]);   // S buffer may be overwritten now
+        // masked scaled scores (log2 domain) and tile max; the mask is warp-uniform
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (mk[c] == 0xFFFFFFFFu) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              sv[c][e] *= sl2;
+              mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              sv[c][e] = ((mk[c] >> e) & 1u) ? sv[c][e] * sl2 : -INFINITY;
+              mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
+            }
+          }
+        }
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        float alpha = 1.f;
+        if (mt > m_ref + kRescaleLog2) {   // also taken on the first tile (m_ref = -inf)
+          alpha = ex2_approx(m_ref - mt);
+          m_ref = mt;
+        }
+        // probabilities -> bf16 pairs (key 2j in the low half of column j), row sum
+        float rs2[2] = {0.f, 0.f};
+        uint32_t packed[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2_approx(sv[c][e] - m_ref);
+            const float p1 = ex2_approx(sv[c][e + 1] - m_ref);
+            rs2[0] += p0;
+            rs2[1] += p1;
+            packed[c][e >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        if (t >= 1) {  // PV(t-1) must be done before P and O are touched
+          if (!attn_warp_wait(B, &B->o_full, pv_iter & 1, ns, SITE_ATTN_SOFTMAX)) { ok = false; break; }
+          tc_fence_after();
+          ++pv_iter;
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {   // rescale O rows in TMEM
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              float ov[32];
+              tmem_ld32_sync(o_addr + c * 32, ov);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+              tmem_st32(o_addr + c * 32, ov);
+            }
+            tmem_st_wait();
+          }
+        }
+        l = l * alpha + (rs2[0] + rs2[1]);
+        tmem_st64(tmem + lane_off + Cfg::TM_P, reinterpret_cast<const uint32_t(&)[64]>(packed));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->p_full);
+      }
+      if (!ok) break;
+      if (ntk > 0) {
+        if (!attn_warp_wait(B, &B->o_full, pv_iter & 1, ns, SITE_ATTN_SOFTMAX)) break;
+        tc_fence_after();
+        ++pv_iter;
+        const float inv = 1.f / l;
+        const size_t grow = static_cast<size_t>(it.h) * P.N + it.q0 + row;
+        uint4 *dst = reinterpret_cast<uint4 *>(P.op + grow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float ov[32];
+          tmem_ld32_sync(o_addr + c * 32, ov);
+          if (row < nrows) {
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8)
+              dst[c * 4 + v8] = make_uint4(pack_bf16x2(ov[8 * v8] * inv, ov[8 * v8 + 1] * inv),
+                                           pack_bf16x2(ov[8 * v8 + 2] * inv, ov[8 * v8 + 3] * inv),
+                                           pack_bf16x2(ov[8 * v8 + 4] * inv, ov[8 * v8 + 5] * inv),
+                                           pack_bf16x2(ov[8 * v8 + 6] * inv, ov[8 * v8 + 7] * inv));
+          }
+        }
+        tc_fence_before();
+        if (row < nrows && P.lse) P.lse[grow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ planning
+// Per (head, q-cluster): number of 128-row q-tiles and of 128-key tiles.
+__global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
+                                       const int32_t *__restrict__ k_off,
+                                       const int32_t *__restrict__ sel_count,
+                                       const int32_t *__restrict__ sel_cols, int BH, int Cq, int Ck,
+                                       int32_t *__restrict__ qtiles, int32_t *__restrict__ ktiles) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= BH * Cq) return;
+  const int h = idx / Cq, i = idx % Cq;
+  const int nq = q_off[h * (Cq + 1) + i + 1] - q_off[h * (Cq + 1) + i];
+  const int cnt = sel_count[idx];
+  const int32_t *cols = sel_cols + static_cast<size_t>(idx) * Ck;
+  const int32_t *ko = k_off + static_cast<size_t>(h) * (Ck + 1);
+  int slots = 0;
+  for (int c = 0; c < cnt; ++c) {
+    const int j = cols[c];
+    if (j < 0 || j >= Ck) {
+      record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
+      continue;
+    }
+    slots += (ko[j + 1] - ko[j] + 7) >> 3;
+  }
+  int qt = nq > 0 ? (nq + 127) >> 7 : 0;
+  if (qt > 0 && slots == 0) {
+    record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
+    qt = 0;
+  }
+  qtiles[idx] = qt;
+  ktiles[idx] = (slots + 15) >> 4;
+}
+
+// Single block: exclusive scan of q-tile counts, then one AttnItem per q-tile.
+__global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
+    const int32_t *__restrict__ q_off, const int32_t *__restrict__ qtiles,
+    const int32_t *__restrict__ ktiles, int BH, int Cq, AttnItem *__restrict__ items,
+    int32_t *__restrict__ num_items) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int total = BH * Cq;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int base = 0; base < total; base += 1024) {
+    const int idx = base + threadIdx.x;
+    const int v = idx < total ? qtiles[idx] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      const int t = warp_tot[lane];
+      int ti = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) ti += y;
+      }
+      warp_tot[lane] = ti - t;
+    }
+    __syncthreads();
+    const int start = carry + warp_tot[w] + incl - v;
+    if (idx < total && v > 0) {
+      const int h = idx / Cq, i = idx % Cq;
+      const int r0 = q_off[h * (Cq + 1) + i], r1 = q_off[h * (Cq + 1) + i + 1];
+      const int kt = ktiles[idx];
+      for (int t = 0; t < v; ++t) {
+        const int q0 = r0 + t * 128;
+        const int rows = min(128, r1 - q0);
+        items[start + t] = AttnItem{h, i, q0, rows | (kt << 8)};
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) carry = start + v;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *num_items = carry;
+}
+
+}  // namespace svg

@@ -1,0 +1,394 @@
+// libsvg.so: host side of the C ABI declared in include/svg.h.
+// One translation unit, so every kernel shares one device error word.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "kmeans.cuh"
+#include "kmeans_tc.cuh"
+#include "select.cuh"
+#include "sort.cuh"
+
+using namespace svg;
+
+namespace {
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+uint64_t g_wait_ns = kDefaultWaitNs;
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline svg_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SVG_OK;
+  return SVG_ERR_CUDA;
+}
+
+inline svg_status launch_status() { return cuda_status(cudaGetLastError()); }
+
+// --------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D view [rows, D] of a bf16 tensor; boxes of 64 channels x box_rows rows,
+// 128-byte swizzle (the tcgen05 K-major / MN-major canonical layout).
+bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, int D, int box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int g_num_sms = 0;
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+template <typename F>
+bool set_smem(F kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes)) == cudaSuccess;
+}
+
+// --------------------------------------------------------------- workspace carving
+struct Carve {
+  uint8_t *p;
+  size_t used = 0;
+  template <typename T>
+  T *take(size_t count) {
+    T *r = reinterpret_cast<T *>(p ? p + used : nullptr);
+    used += align256(count * sizeof(T));
+    return r;
+  }
+};
+
+inline int kmeans_cpad(int C) { return (C + KmCfg<128>::NC - 1) / KmCfg<128>::NC * KmCfg<128>::NC; }
+
+struct KmeansWs {
+  double *sums;
+  float *norms;
+  __nv_bfloat16 *hi, *lo;
+  int32_t *perm, *offsets, *chunk;
+};
+KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
+  Carve c{static_cast<uint8_t *>(ws)};
+  KmeansWs w;
+  const size_t cp = static_cast<size_t>(BH) * kmeans_cpad(C);
+  w.sums = c.take<double>(static_cast<size_t>(BH) * C * D);
+  w.norms = c.take<float>(cp);
+  w.hi = c.take<__nv_bfloat16>(cp * D);
+  w.lo = c.take<__nv_bfloat16>(cp * D);
+  w.perm = c.take<int32_t>(static_cast<size_t>(BH) * N);
+  w.offsets = c.take<int32_t>(static_cast<size_t>(BH) * (C + 1));
+  w.chunk = c.take<int32_t>(static_cast<size_t>(BH) * num_chunks(N) * C);
+  *bytes = c.used;
+  return w;
+}
+
+struct AttnWs {
+  int32_t *num_items, *qtiles, *ktiles;
+  AttnItem *items;
+};
+AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
+  Carve c{static_cast<uint8_t *>(ws)};
+  AttnWs w;
+  w.num_items = c.take<int32_t>(1);
+  w.qtiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
+  w.ktiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
+  w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + 127) / 128 + Cq));
+  *bytes = c.used;
+  return w;
+}
+
+bool sizes_ok(int BH, int N) {
+  return BH > 0 && N > 0 && static_cast<int64_t>(BH) * N < (1ll << 31) - 1;
+}
+
+// Stable counting sort of assign[BH,N] by cluster: perm, offsets (and counts).
+svg_status run_sort(const int32_t *assign, int BH, int N, int C, int32_t *perm, int32_t *offsets,
+                    int32_t *counts, int32_t *chunk, cudaStream_t s) {
+  const int nch = num_chunks(N);
+  sort_hist_kernel<<<dim3(nch, BH), 256, 0, s>>>(assign, N, C, chunk);
+  sort_scan_kernel<<<BH, 1024, 0, s>>>(chunk, N, C, nch, offsets, counts);
+  sort_scatter_kernel<<<dim3(nch, BH), 32, 0, s>>>(assign, N, C, chunk, perm);
+  return launch_status();
+}
+
+svg_status run_row_move(bool gather, int ntensors, const void *const *src, void *const *dst,
+                        const int32_t *perm, int BH, int N, int D, cudaStream_t s) {
+  RowMoveArgs a{};
+  for (int t = 0; t < ntensors; ++t) {
+    a.src[t] = static_cast<const uint4 *>(src[t]);
+    a.dst[t] = static_cast<uint4 *>(dst[t]);
+  }
+  const int vpr = D / 8;
+  const size_t total = static_cast<size_t>(BH) * N * vpr;
+  const size_t per_block = 256 * kVecPerThread;
+  size_t blocks = (total + per_block - 1) / per_block;
+  const size_t cap = static_cast<size_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks == 0) blocks = 1;
+  if (gather)
+    row_move_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, ntensors, perm, BH, N,
+                                                                        vpr);
+  else
+    row_move_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, ntensors, perm, BH, N,
+                                                                         vpr);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *svg_status_string(svg_status s) {
+  switch (s) {
+    case SVG_OK: return "SVG_OK";
+    case SVG_ERR_INVALID_ARG: return "SVG_ERR_INVALID_ARG";
+    case SVG_ERR_UNSUPPORTED: return "SVG_ERR_UNSUPPORTED";
+    case SVG_ERR_WORKSPACE: return "SVG_ERR_WORKSPACE";
+    case SVG_ERR_CUDA: return "SVG_ERR_CUDA";
+    case SVG_ERR_TIMEOUT: return "SVG_ERR_TIMEOUT";
+    case SVG_ERR_DEVICE_CHECK: return "SVG_ERR_DEVICE_CHECK";
+  }
+  return "SVG_ERR_UNKNOWN";
+}
+
+const char *svg_version(void) { return "svg-b200 0.1 (sm_100a)"; }
+
+void svg_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
+
+svg_status svg_get_error(svg_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SVG_ERR_CUDA;
+  uint32_t word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return SVG_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return SVG_ERR_CUDA;
+  return static_cast<svg_status>(word & 0xFFu);
+}
+
+// ------------------------------------------------------------------ k-means
+size_t svg_kmeans_workspace_size(int BH, int N, int D, int C) {
+  if (!sizes_ok(BH, N) || C <= 0 || D <= 0) return 0;
+  size_t bytes = 0;
+  carve_kmeans(nullptr, BH, N, D, C, &bytes);
+  return bytes;
+}
+
+svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, float *centroids,
+                      int32_t *assign, int32_t *counts, void *ws, size_t ws_bytes,
+                      svg_stream_t stream) {
+  if (!x || !centroids || !assign || !counts || !ws) return SVG_ERR_INVALID_ARG;
+  if (!sizes_ok(BH, N) || C < 1 || C > N || iters < 1) return SVG_ERR_INVALID_ARG;
+  if (C > kMaxClusters) return SVG_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(centroids, 16) || !aligned(ws, 256)) return SVG_ERR_INVALID_ARG;
+  size_t need = 0;
+  KmeansWs w = carve_kmeans(ws, BH, N, D, C, &need);
+  if (ws_bytes < need) return SVG_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  const int Cpad = kmeans_cpad(C);
+  CUtensorMap mx, mhi, mlo;
+  if (!make_map_bf16(&mx, x, static_cast<uint64_t>(BH) * N, D, 128) ||
+      !make_map_bf16(&mhi, w.hi, static_cast<uint64_t>(BH) * Cpad, D, 128) ||
+      !make_map_bf16(&mlo, w.lo, static_cast<uint64_t>(BH) * Cpad, D, 128))
+    return SVG_ERR_CUDA;
+  kmeans_split_kernel<<<dim3((Cpad + 7) / 8, BH), 256, 0, s>>>(centroids, C, Cpad, D, w.hi, w.lo,
+                                                              w.norms, w.sums);
+  const dim3 ga((N + 127) / 128, BH);
+  const dim3 gu((C + 7) / 8, BH);
+  const int segs = (N + kAccumRowsPerWarp - 1) / kAccumRowsPerWarp;
+  const dim3 gacc((segs + 7) / 8, BH);
+  if (D == 128) {
+    if (!set_smem(kmeans_assign_tc_kernel<128>, KmCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
+  } else {
+    if (!set_smem(kmeans_assign_tc_kernel<64>, KmCfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
+  }
+  for (int it = 0; it < iters; ++it) {
+    if (D == 128)
+      kmeans_assign_tc_kernel<128><<<ga, KmCfg<128>::THREADS, KmCfg<128>::SMEM_BYTES, s>>>(
+          mx, mhi, mlo, N, C, Cpad, w.norms, centroids, assign, g_wait_ns);
+    else
+      kmeans_assign_tc_kernel<64><<<ga, KmCfg<64>::THREADS, KmCfg<64>::SMEM_BYTES, s>>>(
+          mx, mhi, mlo, N, C, Cpad, w.norms, centroids, assign, g_wait_ns);
+    svg_status st = run_sort(assign, BH, N, C, w.perm, w.offsets, counts, w.chunk, s);
+    if (st != SVG_OK) return st;
+    if (D == 128) {
+      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, assign, w.sums);
+      kmeans_finalize_kernel<128><<<gu, 256, 0, s>>>(C, Cpad, w.offsets, w.sums, centroids, w.hi,
+                                                     w.lo, w.norms);
+    } else {
+      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, assign, w.sums);
+      kmeans_finalize_kernel<64><<<gu, 256, 0, s>>>(C, Cpad, w.offsets, w.sums, centroids, w.hi,
+                                                    w.lo, w.norms);
+    }
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ permutation
+size_t svg_permute_workspace_size(int BH, int N, int C) {
+  if (!sizes_ok(BH, N) || C <= 0) return 0;
+  return align256(static_cast<size_t>(BH) * num_chunks(N) * C * sizeof(int32_t));
+}
+
+svg_status svg_permute(const int32_t *assign, int BH, int N, int C, int32_t *perm,
+                       int32_t *offsets, int ntensors, const void *const *src, void *const *dst,
+                       int D, void *ws, size_t ws_bytes, svg_stream_t stream) {
+  if (!assign || !perm || !offsets || !ws) return SVG_ERR_INVALID_ARG;
+  if (!sizes_ok(BH, N) || C < 1 || ntensors < 0 || ntensors > 3) return SVG_ERR_INVALID_ARG;
+  if (C > kMaxClusters) return SVG_ERR_UNSUPPORTED;
+  if (ntensors > 0) {
+    if (!src || !dst) return SVG_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+    for (int t = 0; t < ntensors; ++t) {
+      if (!src[t] || !dst[t] || !aligned(src[t], 16) || !aligned(dst[t], 16))
+        return SVG_ERR_INVALID_ARG;
+      if (src[t] == dst[t]) return SVG_ERR_INVALID_ARG;
+    }
+  }
+  if (!aligned(ws, 256)) return SVG_ERR_INVALID_ARG;
+  if (ws_bytes < svg_permute_workspace_size(BH, N, C)) return SVG_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  svg_status st = run_sort(assign, BH, N, C, perm, offsets, nullptr, static_cast<int32_t *>(ws), s);
+  if (st != SVG_OK || ntensors == 0) return st;
+  return run_row_move(true, ntensors, src, dst, perm, BH, N, D, s);
+}
+
+svg_status svg_unpermute(const void *xp, const int32_t *perm, int BH, int N, int D, void *x,
+                         svg_stream_t stream) {
+  if (!xp || !perm || !x || xp == x) return SVG_ERR_INVALID_ARG;
+  if (!sizes_ok(BH, N)) return SVG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (!aligned(xp, 16) || !aligned(x, 16)) return SVG_ERR_INVALID_ARG;
+  const void *src[1] = {xp};
+  void *dst[1] = {x};
+  return run_row_move(false, 1, src, dst, perm, BH, N, D, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ top-p selection
+svg_status svg_select_topp(const float *mu_q, const int32_t *n_q, const float *mu_k,
+                           const int32_t *n_k, int BH, int Cq, int Ck, int D, float p, float scale,
+                           int32_t *sel_count, int32_t *sel_cols, svg_stream_t stream) {
+  if (!mu_q || !n_q || !mu_k || !n_k || !sel_count || !sel_cols) return SVG_ERR_INVALID_ARG;
+  if (BH <= 0 || Cq <= 0 || Ck <= 0 || !(p > 0.f) || std::isnan(p)) return SVG_ERR_INVALID_ARG;
+  if (Ck > kMaxCk || (D != 64 && D != 128)) return SVG_ERR_UNSUPPORTED;
+  if (!aligned(mu_q, 16) || !aligned(mu_k, 16)) return SVG_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) scale = 1.f / std::sqrt(static_cast<float>(D));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = select_smem_bytes(D, Ck);
+  const dim3 grid((Cq + kRowsPerBlock - 1) / kRowsPerBlock, BH);
+  if (D == 128) {
+    if (!set_smem(select_topp_kernel<128>, smem)) return SVG_ERR_CUDA;
+    select_topp_kernel<128><<<grid, 256, smem, s>>>(mu_q, n_q, mu_k, n_k, Cq, Ck, p, scale,
+                                                    sel_count, sel_cols);
+  } else {
+    if (!set_smem(select_topp_kernel<64>, smem)) return SVG_ERR_CUDA;
+    select_topp_kernel<64><<<grid, 256, smem, s>>>(mu_q, n_q, mu_k, n_k, Cq, Ck, p, scale,
+                                                   sel_count, sel_cols);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ sparse attention
+size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq) {
+  if (!sizes_ok(BH, N) || Cq <= 0) return 0;
+  size_t bytes = 0;
+  carve_attn(nullptr, BH, N, Cq, &bytes);
+  return bytes;
+}
+
+svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
+                           const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
+                           const int32_t *sel_count, const int32_t *sel_cols, float scale,
+                           void *op, float *lse, void *ws, size_t ws_bytes,
+                           svg_stream_t stream) {
+  if (!qp || !kp || !vp || !q_off || !k_off || !sel_count || !sel_cols || !op || !ws)
+    return SVG_ERR_INVALID_ARG;
+  if (!sizes_ok(BH, N) || Cq < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16) ||
+      !aligned(ws, 256))
+    return SVG_ERR_INVALID_ARG;
+  size_t need = 0;
+  AttnWs w = carve_attn(ws, BH, N, Cq, &need);
+  if (ws_bytes < need) return SVG_ERR_WORKSPACE;
+  if (!(scale > 0.f)) scale = 1.f / std::sqrt(static_cast<float>(D));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  const int pairs = BH * Cq;
+  attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
+                                                            Cq, Ck, w.qtiles, w.ktiles);
+  attn_plan_emit_kernel<<<1, 1024, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, w.items,
+                                           w.num_items);
+  svg_status st = launch_status();
+  if (st != SVG_OK) return st;
+
+  AttnMaps maps;
+  const uint64_t rows = static_cast<uint64_t>(BH) * N;
+  if (!make_map_bf16(&maps.q, qp, rows, D, 128)) return SVG_ERR_CUDA;
+  for (int b = 0; b < kNumBoxSizes; ++b)
+    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b) ||
+        !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
+      return SVG_ERR_CUDA;
+  AttnParams prm;
+  prm.q_off = q_off;
+  prm.k_off = k_off;
+  prm.sel_count = sel_count;
+  prm.sel_cols = sel_cols;
+  prm.items = w.items;
+  prm.num_items = w.num_items;
+  prm.op = static_cast<__nv_bfloat16 *>(op);
+  prm.lse = lse;
+  prm.N = N;
+  prm.Cq = Cq;
+  prm.Ck = Ck;
+  prm.BH = BH;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.wait_ns = g_wait_ns;
+  const int grid = num_sms();
+  if (D == 128) {
+    using Cfg = AttnCfg<128>;
+    if (!set_smem(sparse_attn_kernel<128>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
+    sparse_attn_kernel<128><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
+  } else {
+    using Cfg = AttnCfg<64>;
+    if (!set_smem(sparse_attn_kernel<64>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
+    sparse_attn_kernel<64><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
+  }
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/svg.h declares, and rejects bad arguments on the host before any
+launch (these calls return before touching the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_long_svg_b200 as svg
+from sparse_attention_long_svg_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return svg.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "svg.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(svg_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_stages():
+    names = declared_functions()
+    for stage in ("svg_kmeans", "svg_permute", "svg_select_topp", "svg_sparse_attn", "svg_unpermute"):
+        assert stage in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in svg.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings(lib):
+    for code, name in svg.STATUS.items():
+        assert lib.svg_status_string(code).decode() == name
+    assert lib.svg_version().decode().startswith("svg-b200")
+
+
+def test_workspace_sizes_are_positive_and_monotone(lib):
+    a = lib.svg_kmeans_workspace_size(40, 32760, 128, 500)
+    b = lib.svg_kmeans_workspace_size(40, 75600, 128, 1000)
+    assert 0 < a < b
+    assert lib.svg_permute_workspace_size(1, 2048, 64) > 0
+    assert lib.svg_sparse_attn_workspace_size(40, 32760, 100) > 0
+    assert lib.svg_kmeans_workspace_size(0, 10, 64, 4) == 0
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+FAKE = 0x10000  # 256-byte aligned, never dereferenced: every call below fails its host checks
+
+
+def test_invalid_arguments_are_rejected_before_launch(lib):
+    nul = _p(0)
+    f = _p(FAKE)
+    # k-means: null pointer, C > N, iters < 1, unsupported D, too many clusters, small workspace
+    assert lib.svg_kmeans(nul, 1, 16, 64, 4, 1, f, f, f, f, 1 << 20, nul) == 1
+    assert lib.svg_kmeans(f, 1, 16, 64, 17, 1, f, f, f, f, 1 << 20, nul) == 1
+    assert lib.svg_kmeans(f, 1, 16, 64, 4, 0, f, f, f, f, 1 << 20, nul) == 1
+    assert lib.svg_kmeans(f, 1, 16, 96, 4, 1, f, f, f, f, 1 << 20, nul) == 2
+    assert lib.svg_kmeans(f, 1, 4096, 64, 2000, 1, f, f, f, f, 1 << 30, nul) == 2
+    assert lib.svg_kmeans(f, 1, 4096, 64, 64, 1, f, f, f, f, 16, nul) == 3
+    # misaligned bf16 pointer
+    assert lib.svg_kmeans(_p(FAKE + 2), 1, 16, 64, 4, 1, f, f, f, f, 1 << 20, nul) == 1
+    # permute: more than 3 tensors, aliasing src == dst
+    assert lib.svg_permute(f, 1, 16, 4, f, f, 4, f, f, 64, f, 1 << 20, nul) == 1
+    ptrs = (ctypes.c_void_p * 1)(FAKE)
+    arr = ctypes.cast(ptrs, ctypes.c_void_p)
+    assert lib.svg_permute(f, 1, 16, 4, f, f, 1, arr, arr, 64, f, 1 << 20, nul) == 1
+    # select: p <= 0, NaN p, Ck too large
+    assert lib.svg_select_topp(f, f, f, f, 1, 4, 8, 64, 0.0, 0.0, f, f, nul) == 1
+    assert lib.svg_select_topp(f, f, f, f, 1, 4, 8, 64, float("nan"), 0.0, f, f, nul) == 1
+    assert lib.svg_select_topp(f, f, f, f, 1, 4, 2048, 64, 0.9, 0.0, f, f, nul) == 2
+    # attention: unsupported D, workspace too small
+    assert lib.svg_sparse_attn(f, f, f, 1, 16, 80, f, 2, f, 2, f, f, 0.0, f, nul, f, 1 << 20, nul) == 2
+    assert lib.svg_sparse_attn(f, f, f, 1, 4096, 64, f, 2, f, 2, f, f, 0.0, f, nul, f, 8, nul) == 3
+    # unpermute: aliasing
+    assert lib.svg_unpermute(f, f, 1, 16, 64, f, nul) == 1
