@@ -1,0 +1,440 @@
+"""Benchmark of the semantic-aware top-p sparse attention layer on B200.
+
+One step = one pass of the whole hot path over one layer of synthetic
+input: k-means of Q and of K from the seeded token-sampled centroids,
+permutation of Q and of K/V, centroid top-p selection, block-sparse
+attention and un-permutation (the stages of the Sparse VideoGen2 page,
+section 2).  Default workload: 480p, 5 s clip = 32,760 latent tokens
+(21x30x52), 40 heads, head dim 128, 100/500 clusters, 5 k-means rounds,
+top-p 0.9.
+
+Prints ONE JSON line (rank 0).  value = whole-job throughput in effective
+TFLOP/s: algorithmic attention FLOPs on the selected blocks
+(4 * D * sum over selected (q-cluster, k-cluster) pairs of n_q * n_k) of all
+layers processed by all ranks, divided by the max-over-ranks device time of
+the timed steps; ms_per_step is ms per layer.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl svg|reference]
+
+Multi-GPU (one process per GPU, torchrun): every rank runs its own layer
+(heads are independent problems), no collective on the data path; the only
+collectives are the timing barrier and the max-over-ranks reduction.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "ms/layer & effective TFLOPS (% bf16 peak) of top-p sparse attn, 32.7K tok"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks (identity on one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"svg_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [d.get("num_threads", 0) for d in info if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(wl, heads: int):
+    """Runs the oracle on the first `heads` heads; returns (seconds, attention FLOPs)."""
+    from oracle import svg_oracle as so
+    L = synth.make_layer(wl, heads=heads)
+    D = L.q.shape[2]
+    flops = 0.0
+    t0 = time.perf_counter()
+    for h in range(heads):
+        r = so.svg_head(L.q[h], L.k[h], L.v[h], L.init_centroids("q")[h], L.init_centroids("k")[h],
+                        wl.iters, wl.top_p[0])
+        pairs, _ = so.density(r.q_off, r.k_off, [s.cols for s in r.selection])
+        flops += 4.0 * D * pairs
+    return time.perf_counter() - t0, flops
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    heads = 1
+    for _ in range(args.warmup):
+        oracle_sample(wl, heads)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        s, f = oracle_sample(wl, heads)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    sample = f"{heads} of {wl.heads} heads of the {wl.name} layer per step, whole path (k-means, permute, select, attention)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, n_gpus):
+    return {"workload": wl.name, "heads": wl.heads, "tokens": wl.tokens, "grid": list(wl.grid),
+            "head_dim": wl.head_dim, "cq": wl.cq, "ck": wl.ck, "kmeans_iters": wl.iters, "top_p": wl.top_p[0],
+            "layers_per_step_per_gpu": 1, "parallelism": f"dp{n_gpus} (independent layers per GPU)",
+            "l2": "inputs larger than L2 (Q/K/V bf16 = %.0f MB > 126 MB); no flush" %
+                  (3 * wl.heads * wl.tokens * wl.head_dim * 2 / 1e6)}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def kernel_launches_per_step(wl) -> int:
+    """Our kernels per step (counted from the launch sequence in svg.cu)."""
+    per_kmeans = 1 + 6 * wl.iters            # split + T x (assign, hist, scan, scatter, accum, finalize)
+    per_permute = 3 + 1                      # hist, scan, scatter + row gather
+    return 2 * per_kmeans + 2 * per_permute + 1 + 3 + 1   # select; plan x2 + attention; unpermute
+
+
+def attention_pairs(layer, wl):
+    cnt = layer.sel_count.cpu().numpy()
+    cols = layer.sel_cols.cpu().numpy()
+    q_off = layer.q_off.cpu().numpy()
+    k_off = layer.k_off.cpu().numpy()
+    pairs = 0
+    for h in range(cnt.shape[0]):
+        nq = np.diff(q_off[h])
+        nk = np.diff(k_off[h])
+        for i in range(cnt.shape[1]):
+            if cnt[h, i]:
+                pairs += int(nq[i]) * int(nk[cols[h, i, :cnt[h, i]]].sum())
+    return pairs
+
+
+def run_svg(args, wl):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+
+    import sparse_attention_long_svg_b200 as svg
+    svg.load_library()
+    peaks, peak_kind = load_peaks()
+
+    L = synth.make_layer(wl)
+    BH, N, D = L.q.shape
+
+    def to_dev(x):
+        return torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(device)
+
+    q, k, v = to_dev(L.q), to_dev(L.k), to_dev(L.v)
+    mu_q0 = torch.from_numpy(L.init_centroids("q")).to(device)
+    mu_k0 = torch.from_numpy(L.init_centroids("k")).to(device)
+    mu_q, mu_k = mu_q0.clone(), mu_k0.clone()
+    layer = svg.SvgLayer(BH, N, D, wl.cq, wl.ck, device)
+    out = torch.empty_like(q)
+    p = wl.top_p[0]
+    stream = torch.cuda.current_stream()
+    stage_names = ["kmeans_q", "kmeans_k", "permute", "select", "attn", "unpermute"]
+
+    def step(ev=None):
+        mu_q.copy_(mu_q0)
+        mu_k.copy_(mu_k0)
+        if ev:
+            ev[0].record()
+        svg.kmeans(q, mu_q, wl.iters, layer.assign_q, layer.n_q, layer.workspace)
+        if ev:
+            ev[1].record()
+        svg.kmeans(k, mu_k, wl.iters, layer.assign_k, layer.n_k, layer.workspace)
+        if ev:
+            ev[2].record()
+        svg.permute(layer.assign_q, wl.cq, [q], [layer.qp], layer.perm_q, layer.q_off, layer.workspace)
+        svg.permute(layer.assign_k, wl.ck, [k, v], [layer.kp, layer.vp], layer.perm_k, layer.k_off,
+                    layer.workspace)
+        if ev:
+            ev[3].record()
+        svg.select_topp(mu_q, layer.n_q, mu_k, layer.n_k, p, 0.0, layer.sel_count, layer.sel_cols)
+        if ev:
+            ev[4].record()
+        svg.sparse_attn(layer.qp, layer.kp, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
+                        layer.sel_cols, 0.0, layer.op, workspace=layer.workspace)
+        if ev:
+            ev[5].record()
+        svg.unpermute(layer.op, layer.perm_q, out)
+        if ev:
+            ev[6].record()
+
+    clocks = ClockSampler(device.index)
+    clocks.__enter__()          # sampling starts with the warm-up so short runs still see load
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if svg.get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if True:
+        t_start.record()
+        for s in range(args.steps):
+            step(events[s])
+        t_end.record()
+        torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
+    if world > 1:
+        torch.distributed.barrier()
+    local_ms = t_start.elapsed_time(t_end)
+    if svg.get_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    stage_ms = {n: statistics.mean(events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps))
+                for i, n in enumerate(stage_names)}
+
+    pairs = attention_pairs(layer, wl)
+    flops_layer = 4.0 * D * pairs
+    density = pairs / (BH * N * N)
+
+    total_ms = reduce_max(local_ms, world, device)
+    all_flops = reduce_sum(flops_layer * args.steps, world, device)
+    value = all_flops / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), H2D + D2H inside the timed region
+    e2e_steps = max(1, min(args.steps, 3))
+    hq = torch.from_numpy(synth.bf16_bits(L.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(synth.bf16_bits(L.k).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(synth.bf16_bits(L.v).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hmq, hmk = mu_q0.cpu().pin_memory(), mu_k0.cpu().pin_memory()
+    hout = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        mu_q.copy_(hmq, non_blocking=True)
+        mu_k.copy_(hmk, non_blocking=True)
+        o, _ = layer(dq, dk, dv, mu_q, mu_k, wl.iters, p, 0.0, out)
+        hout.copy_(o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, device)
+    e2e_value = reduce_sum(flops_layer * e2e_steps, world, device) / (e2e_ms * 1e-3) / 1e12
+    h2d = int(3 * hq.numel() * 2 + 2 * hmq.numel() * 4)
+    d2h = int(hout.numel() * 2)
+
+    # ---- rooflines
+    tc_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    attn_tflops = flops_layer / (stage_ms["attn"] * 1e-3) / 1e12
+    traffic = load_traffic("sparse_attn_kernel", wl.name)
+    roofline = {"kernel": f"sparse_attn_kernel<{D}>", "bound": "tensor", "achieved": attn_tflops,
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_tflops / tc_peak, "traffic": traffic,
+                "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a multi-ms step)",
+                "algorithmic": "4*D*sum_selected(n_q*n_k) FLOP per launch = %.4g" % flops_layer}
+    tensor_bytes = BH * N * D * 2
+    km_flops = {c: 2.0 * N * c * D * BH * wl.iters for c in (wl.cq, wl.ck)}
+    km_bytes = 2.0 * tensor_bytes * wl.iters          # assign read + update read per round
+    stages = {
+        "kmeans_q": {"ms": stage_ms["kmeans_q"], "tflops": km_flops[wl.cq] / stage_ms["kmeans_q"] / 1e9,
+                     "gbs": km_bytes / stage_ms["kmeans_q"] / 1e6},
+        "kmeans_k": {"ms": stage_ms["kmeans_k"], "tflops": km_flops[wl.ck] / stage_ms["kmeans_k"] / 1e9,
+                     "gbs": km_bytes / stage_ms["kmeans_k"] / 1e6},
+        "permute": {"ms": stage_ms["permute"], "gbs": 6.0 * tensor_bytes / stage_ms["permute"] / 1e6},
+        "select": {"ms": stage_ms["select"]},
+        "attn": {"ms": stage_ms["attn"], "tflops": attn_tflops},
+        "unpermute": {"ms": stage_ms["unpermute"], "gbs": 2.0 * tensor_bytes / stage_ms["unpermute"] / 1e6},
+    }
+    for sname in ("kmeans_q", "kmeans_k", "permute", "unpermute"):
+        stages[sname]["hbm_frac"] = stages[sname]["gbs"] / hbm_peak
+    for sname in ("kmeans_q", "kmeans_k", "attn"):
+        stages[sname]["tensor_frac"] = stages[sname]["tflops"] / tc_peak
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nh = 2
+        secs, fl = oracle_sample(wl, nh)
+        cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{nh} of {wl.heads} heads of the {wl.name} layer, whole path, {secs:.1f} s"}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wl, world),
+            "attn_ms": stage_ms["attn"], "attn_eff_tflops": attn_tflops,
+            "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": kernel_launches_per_step(wl) * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    entry = d.get(kernel, {}).get(workload)
+    if not entry:
+        return None
+    from sparse_attention_long_svg_b200 import build
+    if entry.get("source_hash") != build.source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="480p-5s", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="svg", choices=["svg", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_svg(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -28,6 +28,17 @@ def sources():
     return sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
 
 
+def source_hash() -> str:
+    """Hash of every CUDA source and the ABI header (identifies a kernel build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for path in sources() + [os.path.join(os.path.dirname(HERE), "include", "svg.h")]:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def up_to_date() -> bool:
     if not os.path.exists(OUT):
         return False
