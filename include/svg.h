@@ -146,6 +146,38 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
                            const int32_t *sel_count, const int32_t *sel_cols, float scale, void *op,
                            float *lse, void *ws, size_t ws_bytes, svg_stream_t stream);
 
+/* ------------------------------------------------------------------------ sparse attention, no allocation
+ * No counterpart on the pages: this is a service for callers that cannot hand
+ * the library a scratch buffer.  Some callers have no way to obtain device
+ * memory at the point where they call: a plug-in running inside a host
+ * framework that owns every allocation, an inference loop whose memory budget
+ * is fixed when it starts, or a runtime that forbids device allocation after
+ * initialisation.  This call takes the same inputs and outputs as
+ * svg_sparse_attn and computes the same result, but its scratch space is a
+ * fixed array compiled into the library (SVG_NOALLOC_SCRATCH_BYTES, 2 MiB) that
+ * every GPU which loads the library holds until the process exits.
+ *
+ *  - Limit: svg_sparse_attn_workspace_size(BH, N, Cq), about
+ *    16*BH*(ceil(N/128) + Cq) + 8*BH*Cq bytes, must not exceed
+ *    SVG_NOALLOC_SCRATCH_BYTES (e.g. 80 heads x 75,600 tokens x 200 q-clusters
+ *    needs 1.2 MB); larger sizes return SVG_ERR_WORKSPACE before anything is
+ *    launched.
+ *  - It allocates and frees nothing (no cudaMalloc, no cudaFree, no
+ *    allocating library routine).
+ *  - The first call on each device looks up the device address of the array
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array and it keeps the previous call's contents;
+ *    the call rewrites every scratch entry it reads, so nothing needs
+ *    clearing, but calls whose executions overlap on the GPU (different
+ *    streams, or host threads) race on the array: order them on one stream.
+ */
+#define SVG_NOALLOC_SCRATCH_BYTES (2u << 20)
+svg_status svg_sparse_attn_noalloc(const void *qp, const void *kp, const void *vp, int BH, int N,
+                                   int D, const int32_t *q_off, int Cq, const int32_t *k_off,
+                                   int Ck, const int32_t *sel_count, const int32_t *sel_cols,
+                                   float scale, void *op, float *lse, svg_stream_t stream);
+
 /* ------------------------------------------------------------------------ un-permutation
  * Inverse permutation (section 2(a) "Mathematical equivalence"):
  * x[h][perm[h][r]] = xp[h][r] for every row r.  x must not alias xp.

@@ -44,7 +44,10 @@ SIGNATURES = {
     "svg_sparse_attn_workspace_size": (_SZ, [_I, _I, _I]),
     "svg_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "svg_sparse_attn_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P]),
 }
+
+NOALLOC_SCRATCH_BYTES = 2 << 20   # SVG_NOALLOC_SCRATCH_BYTES in include/svg.h
 
 _lib = None
 
@@ -207,6 +210,30 @@ def sparse_attn(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.
     _check("svg_sparse_attn", lib.svg_sparse_attn(
         _ptr(qp), _ptr(kp), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
         _ptr(sel_cols), float(scale), _ptr(op), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return op, lse
+
+
+def sparse_attn_noalloc(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
+                       want_lse: bool = False, lse=None, stream=None):
+    """sparse_attn for callers that cannot provide device scratch memory.
+
+    Same inputs and result as ``sparse_attn``; the library uses a fixed scratch
+    array of its own instead of a workspace (see svg_sparse_attn_noalloc in
+    include/svg.h: size limit, one shared array, calls must not overlap).
+    """
+    lib = load_library()
+    for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
+        _need(t, n, torch.bfloat16, 3)
+    BH, N, D = qp.shape
+    Cq = q_off.shape[1] - 1
+    Ck = k_off.shape[1] - 1
+    if op is None:
+        op = torch.empty_like(qp)
+    if want_lse and lse is None:
+        lse = torch.empty((BH, N), dtype=torch.float32, device=qp.device)
+    _check("svg_sparse_attn_noalloc", lib.svg_sparse_attn_noalloc(
+        _ptr(qp), _ptr(kp), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
+        _ptr(sel_cols), float(scale), _ptr(op), _ptr(lse), _stream(stream)))
     return op, lse
 
 

@@ -392,3 +392,46 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ sparse attention without allocation
+// Scratch for callers that cannot pass a workspace (see svg.h): a fixed array
+// in this module, one per device that loads the library.  Host code must not
+// hand the symbol itself to a kernel (in host code it only names a host-side
+// stand-in); its device address is looked up once per device.
+namespace {
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SVG_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+void *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
+void *noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" svg_status svg_sparse_attn_noalloc(const void *qp, const void *kp, const void *vp, int BH,
+                                              int N, int D, const int32_t *q_off, int Cq,
+                                              const int32_t *k_off, int Ck,
+                                              const int32_t *sel_count, const int32_t *sel_cols,
+                                              float scale, void *op, float *lse,
+                                              svg_stream_t stream) {
+  if (!sizes_ok(BH, N) || Cq < 1) return SVG_ERR_INVALID_ARG;
+  const size_t need = svg_sparse_attn_workspace_size(BH, N, Cq);
+  if (need == 0 || need > SVG_NOALLOC_SCRATCH_BYTES) return SVG_ERR_WORKSPACE;
+  void *ws = noalloc_scratch_address();
+  if (ws == nullptr) return SVG_ERR_CUDA;
+  // Every scratch entry the attention path reads is written earlier in the
+  // same call (planning kernels), so leftovers of a previous call are harmless.
+  return svg_sparse_attn(qp, kp, vp, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale, op,
+                         lse, ws, SVG_NOALLOC_SCRATCH_BYTES, stream);
+}
