@@ -203,7 +203,7 @@ def workload_config(wl, n_gpus):
 
 def kernel_launches_per_step(wl) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
-    per_kmeans = 1 + 6 * wl.iters            # split + T x (assign, hist, scan, scatter, accum, finalize)
+    per_kmeans = 2 + 7 * wl.iters            # split, |x|^2 + T x (assign, refine, hist, scan, scatter, accum, finalize)
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
     return 2 * per_kmeans + 2 * per_permute + 1 + 3 + 1   # select; plan x2 + attention; unpermute
 

@@ -195,6 +195,13 @@ svg_status svg_unpermute(const void *xp, const int32_t *perm, int BH, int N, int
 svg_status svg_get_error(svg_stream_t stream);
 void svg_set_wait_timeout_ns(uint64_t ns);
 
+/* Test hook for failure detection (no GPU fault involved): fault = 1 makes
+ * the following svg_sparse_attn launches skip loading their query tiles, so
+ * the kernel's bounded waits run out, it records SVG_ERR_TIMEOUT, waits for
+ * its own in-flight copies, frees its tensor memory and returns; fault = 0
+ * restores normal operation.  Outputs of a faulted launch are undefined. */
+void svg_debug_set_fault(int fault);
+
 /* Library version, e.g. "svg-b200 0.1 (sm_100a)". */
 const char *svg_version(void);
 

@@ -35,6 +35,7 @@ SIGNATURES = {
     "svg_status_string": (ctypes.c_char_p, [_I]),
     "svg_version": (ctypes.c_char_p, []),
     "svg_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
+    "svg_debug_set_fault": (None, [_I]),
     "svg_get_error": (_I, [_P]),
     "svg_kmeans_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "svg_kmeans": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),

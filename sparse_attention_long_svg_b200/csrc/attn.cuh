@@ -22,10 +22,10 @@
 //   warp 6     item loader: the next q-tile's selected key ranges, read from
 //              global memory into a 2-entry shared-memory ring ahead of time
 // Per key tile k: S(k) -> softmax(k) writes P(k) (bf16 pairs, TMEM) ->
-// PV(k) with A = P read from TMEM.  O accumulates in TMEM across the key tiles of a q-tile; the softmax
-// warps rescale it in place only when a row's running max grows by more than
-// 2^8 (exact: every probability is taken against the same reference max that
-// O and the row sum use).
+// PV(k) with A = P read from TMEM.  O accumulates in TMEM across the key
+// tiles of a q-tile; the softmax warps rescale it in place only when a row's
+// running max grows by more than 2^8 (exact: every probability is taken
+// against the same reference max that O and the row sum use).
 #pragma once
 #include "common.cuh"
 
@@ -108,6 +108,7 @@ struct AttnParams {
   int N, Cq, Ck, BH;
   float scale_log2;      // softmax scale * log2(e)
   uint64_t wait_ns;
+  int fault;             // test hook: 1 = never load the query tile (waits must run out)
 };
 
 __device__ __forceinline__ bool attn_wait(AttnBarriers *b, uint64_t *bar, uint32_t parity,
@@ -228,7 +229,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
-    uint32_t g = 0;  // global key-tile counter
+    uint32_t g = 0;            // global key-tile counter
+    uint32_t nq = 0, gk = 0, gv = 0;  // Q tiles, K tiles and V tiles issued (for the drain)
     int n_items = 0;
     if (lane == 0) {
       bool ok = true;
@@ -241,11 +243,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int ntk = it.packed >> 8;
         if (n_items > 0 && !attn_wait(B, &B->q_empty, (n_items - 1) & 1, ns, SITE_ATTN_PRODUCER))
           break;
-        mbar_arrive_expect_tx(&B->q_full, Cfg::Q_BYTES);
-        const int qrow = it.h * P.N + it.q0;
+        if (P.fault != 1) {
+          mbar_arrive_expect_tx(&B->q_full, Cfg::Q_BYTES);
+          const int qrow = it.h * P.N + it.q0;
 #pragma unroll
-        for (int dh = 0; dh < Cfg::DH; ++dh)
-          tma_load_2d(sQ + dh * Cfg::HALF_Q, &maps.q, dh * 64, qrow, &B->q_full);
+          for (int dh = 0; dh < Cfg::DH; ++dh)
+            tma_load_2d(sQ + dh * Cfg::HALF_Q, &maps.q, dh * 64, qrow, &B->q_full);
+          ++nq;
+        }
         int ci = 0, cur = 0, left = 0;
         const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
         for (int t = 0; t < ntk; ++t, ++g) {
@@ -291,6 +296,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               tma_load_2d(kdst + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64, box_row[bx],
                           &B->k_full[st]);
           }
+          gk = g + 1;
           if (g >= 3 && !attn_wait(B, &B->v_empty[vs], vph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
           B->meta[vs][0] = mask[0];
           B->meta[vs][1] = mask[1];
@@ -306,17 +312,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               tma_load_2d(vdst + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64, box_row[bx],
                           &B->v_full[vs]);
           }
+          gv = g + 1;
         }
         mbar_arrive(&B->item_empty[buf]);   // the ranges of this item are no longer read
       }
       // drain: every load issued above lands on a full barrier; wait for the
       // last phase of each so no copy is in flight when the CTA exits.
       if (aborted(B)) {
-        if (n_items > 0) mbar_wait(&B->q_full, (n_items - 1) & 1, 1000000000ull);
-        for (uint32_t k = (g >= 3 ? g - 3 : 0); k < g; ++k) {
+        if (nq > 0) mbar_wait(&B->q_full, (nq - 1) & 1, 1000000000ull);
+        for (uint32_t k = (gk >= 2 ? gk - 2 : 0); k < gk; ++k)
           mbar_wait(&B->k_full[k & 1], (k >> 1) & 1, 1000000000ull);
+        for (uint32_t k = (gv >= 3 ? gv - 3 : 0); k < gv; ++k)
           mbar_wait(&B->v_full[k % 3], (k / 3) & 1, 1000000000ull);
-        }
       }
     }
   } else if (warp == 5) {

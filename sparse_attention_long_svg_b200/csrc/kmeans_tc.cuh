@@ -6,13 +6,17 @@
 // bf16 high part and a bf16 low part (mu = hi + lo + r, |r| <= 2^-17 |mu|
 // per channel) and x . mu is accumulated as x . hi + x . lo in fp32 TMEM.
 // The epilogue keeps the best two centroids; when they are closer than the
-// tensor-core error allows to separate, the exact float32 distances decide.
+// tensor-core error allows to separate, the token goes on a near-tie list and
+// kmeans_refine_kernel decides it with the exact float32 distances.
 //
-// One CTA per (128-token tile, head), ~97 KB shared memory so two CTAs share
-// an SM.  Warps 0-3: epilogue (thread t = token t of the tile = TMEM lane t);
-// warp 4: TMA producer; warp 5: MMA issuer and TMEM owner.  Centroids stream
-// in chunks of 128 (one smem stage); the two TMEM accumulators let the
-// epilogue of chunk j overlap the MMAs of chunk j+1.
+// Persistent: one CTA per SM walks units (head, 128-token tile) in
+// head-major order (the head's centroids stay hot in L2).  Warps 0-7:
+// epilogue in two groups of four (thread t of a group = token t of the tile
+// = TMEM lane t), taking alternate chunks; warp 8: TMA producer (x tiles,
+// centroid chunks and their squared norms); warp 9: MMA issuer and TMEM
+// owner.  x tiles (2-deep ring) and centroid chunks of 128 (hi and lo parts,
+// 2-deep ring) stream through shared memory; two TMEM accumulators let the
+// epilogue of one chunk overlap the MMAs of the next.
 #pragma once
 #include "common.cuh"
 
@@ -21,21 +25,34 @@ namespace svg {
 template <int D>
 struct KmCfg {
   static constexpr int BM = 128, NC = 128, DH = D / 64;
+  static constexpr int XST = 2, CST = 2;  // x tile ring, centroid chunk ring
   static constexpr int X_BYTES = BM * D * 2, C_BYTES = NC * D * 2;
   static constexpr int HALF = 128 * 128;  // one 64-channel half of a 128-row tile
-  static constexpr int OFF_X = 0, OFF_HI = X_BYTES, OFF_LO = OFF_HI + C_BYTES;
-  static constexpr int OFF_BAR = OFF_LO + C_BYTES;
+  static constexpr int OFF_X = 0;
+  static constexpr int OFF_C = OFF_X + XST * X_BYTES;          // stage: hi part then lo part
+  static constexpr int OFF_NORM = OFF_C + CST * 2 * C_BYTES;   // 2 x NC fp32 squared norms
+  static constexpr int OFF_MERGE = OFF_NORM + 2 * NC * 4;      // 2 x 128 x (best, arg, second, arg2)
+  static constexpr int OFF_BAR = OFF_MERGE + 2 * 128 * 16;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static constexpr uint32_t TM_COLS = 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NC, false, false);
-  static constexpr int THREADS = 192;
+  static constexpr int EPI_WARPS = 8;                          // two groups of four
+  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
+  static constexpr int PRODUCER_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
 };
 
 struct KmBarriers {
-  uint64_t x_full, c_full, c_empty, acc_full[2], acc_empty[2], drain;
+  uint64_t x_full[2], x_empty[2], c_full[2], c_empty[2], acc_full[2], acc_empty[2];
+  uint64_t n_full[2], n_empty[2], merge_full[2], merge_empty[2], drain;
   uint32_t tmem_base;
   int32_t abort_flag;
 };
+
+// One near-tie token: flat token index (h * N + n) and its two candidates.
+struct KmTie {
+  int32_t token, a, b, pad;
+};
+
 
 __device__ __forceinline__ bool km_wait(KmBarriers *b, uint64_t *bar, uint32_t parity, uint64_t ns,
                                         uint32_t site) {
@@ -47,11 +64,12 @@ __device__ __forceinline__ bool km_wait(KmBarriers *b, uint64_t *bar, uint32_t p
 
 // Splits fp32 centroids into bf16 hi/lo parts and squared norms for chunks of
 // NC rows; rows C..Cpad-1 get zero parts and +inf norm (never the argmin).
-// Also clears the fp64 update sums [BH, C, D] for the first round.
+// Also clears the near-tie counter before the first assign step.
 __global__ void kmeans_split_kernel(const float *__restrict__ mu, int C, int Cpad, int D,
                                     __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo,
-                                    float *__restrict__ norms, double *__restrict__ sums) {
+                                    float *__restrict__ norms, int32_t *__restrict__ num_ties) {
   const int h = blockIdx.y;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *num_ties = 0;
   const int c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (c >= Cpad) return;
@@ -64,7 +82,6 @@ __global__ void kmeans_split_kernel(const float *__restrict__ mu, int C, int Cpa
     hi[orow + d] = vh;
     lo[orow + d] = vl;
     s = fmaf(v, v, s);
-    if (c < C) sums[(static_cast<size_t>(h) * C + c) * D + d] = 0.0;
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -72,37 +89,45 @@ __global__ void kmeans_split_kernel(const float *__restrict__ mu, int C, int Cpa
 }
 
 template <int D>
-__global__ void __launch_bounds__(KmCfg<D>::THREADS)
+__global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                             const __grid_constant__ CUtensorMap map_hi,
-                            const __grid_constant__ CUtensorMap map_lo, int N, int C, int Cpad,
-                            const float *__restrict__ norms, const float *__restrict__ mu,
-                            int32_t *__restrict__ assign, uint64_t wait_ns) {
+                            const __grid_constant__ CUtensorMap map_lo, int BH, int N, int C,
+                            int Cpad, const float *__restrict__ norms,
+                            const float *__restrict__ xnorm, int32_t *__restrict__ assign,
+                            KmTie *__restrict__ ties, int32_t *__restrict__ num_ties,
+                            uint64_t wait_ns) {
   using Cfg = KmCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  uint8_t *sX = smem + Cfg::OFF_X;
-  uint8_t *sHi = smem + Cfg::OFF_HI;
-  uint8_t *sLo = smem + Cfg::OFF_LO;
   KmBarriers *B = reinterpret_cast<KmBarriers *>(smem + Cfg::OFF_BAR);
+  float *sNorm = reinterpret_cast<float *>(smem + Cfg::OFF_NORM);
+  float4 *sMerge = reinterpret_cast<float4 *>(smem + Cfg::OFF_MERGE);
   const int warp = static_cast<int>(warp_id()), lane = static_cast<int>(lane_id());
-  const int h = blockIdx.y, n0 = blockIdx.x * Cfg::BM;
+  const int tiles = (N + Cfg::BM - 1) / Cfg::BM;
+  const int units = BH * tiles;              // unit u = (head u / tiles, tile u % tiles)
   const int nchunks = Cpad / Cfg::NC;
+  const int grid = static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    mbar_init(&B->x_full, 1);
-    mbar_init(&B->c_full, 1);
-    mbar_init(&B->c_empty, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&B->x_full[s], 1);
+      mbar_init(&B->x_empty[s], 1);          // released by the MMA commit after a unit
+      mbar_init(&B->c_full[s], 1);
+      mbar_init(&B->c_empty[s], 1);
       mbar_init(&B->acc_full[s], 1);
-      mbar_init(&B->acc_empty[s], 4);
+      mbar_init(&B->acc_empty[s], 4);        // the four warps of the group that read it
+      mbar_init(&B->n_full[s], 1);
+      mbar_init(&B->n_empty[s], 4);
+      mbar_init(&B->merge_full[s], 4);
+      mbar_init(&B->merge_empty[s], 4);
     }
     mbar_init(&B->drain, 1);
     B->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     tmem_alloc(&B->tmem_base, Cfg::TM_COLS);
     tmem_relinquish();
   }
@@ -111,138 +136,274 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS)
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
 
-  if (warp == 4) {
+  if (warp == Cfg::PRODUCER_WARP) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int j = 0;
-      mbar_arrive_expect_tx(&B->x_full, Cfg::X_BYTES);
+      uint32_t nu = 0, gc = 0;   // units and chunks issued by this CTA
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += grid, ++nu) {
+        const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
+        const int xs = nu & 1;
+        if (nu >= 2 && !km_wait(B, &B->x_empty[xs], ((nu >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA)) break;
+        mbar_arrive_expect_tx(&B->x_full[xs], Cfg::X_BYTES);
+        uint8_t *xd = smem + Cfg::OFF_X + xs * Cfg::X_BYTES;
 #pragma unroll
-      for (int dh = 0; dh < Cfg::DH; ++dh)
-        tma_load_2d(sX + dh * Cfg::HALF, &map_x, dh * 64, h * N + n0, &B->x_full);
-      for (; j < nchunks; ++j) {
-        if (j > 0 && !km_wait(B, &B->c_empty, (j - 1) & 1, wait_ns, SITE_KMEANS_MMA)) break;
-        mbar_arrive_expect_tx(&B->c_full, 2 * Cfg::C_BYTES);
-        const int crow = h * Cpad + j * Cfg::NC;
+        for (int dh = 0; dh < Cfg::DH; ++dh)
+          tma_load_2d(xd + dh * Cfg::HALF, &map_x, dh * 64, h * N + n0, &B->x_full[xs]);
+        for (int j = 0; j < nchunks; ++j, ++gc) {
+          const int cs = gc & 1;
+          if (gc >= 2 && (!km_wait(B, &B->c_empty[cs], ((gc >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA) ||
+                          !km_wait(B, &B->n_empty[cs], ((gc >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA))) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&B->c_full[cs], 2 * Cfg::C_BYTES);
+          uint8_t *cd = smem + Cfg::OFF_C + cs * 2 * Cfg::C_BYTES;
+          const int crow = h * Cpad + j * Cfg::NC;
 #pragma unroll
-        for (int dh = 0; dh < Cfg::DH; ++dh) {
-          tma_load_2d(sHi + dh * Cfg::HALF, &map_hi, dh * 64, crow, &B->c_full);
-          tma_load_2d(sLo + dh * Cfg::HALF, &map_lo, dh * 64, crow, &B->c_full);
+          for (int dh = 0; dh < Cfg::DH; ++dh) {
+            tma_load_2d(cd + dh * Cfg::HALF, &map_hi, dh * 64, crow, &B->c_full[cs]);
+            tma_load_2d(cd + Cfg::C_BYTES + dh * Cfg::HALF, &map_lo, dh * 64, crow, &B->c_full[cs]);
+          }
+          mbar_arrive_expect_tx(&B->n_full[cs], Cfg::NC * 4);
+          bulk_load(sNorm + cs * Cfg::NC, norms + static_cast<size_t>(crow), Cfg::NC * 4, &B->n_full[cs]);
         }
       }
-      // drain: the last issued chunk and x must have landed before exit
-      mbar_wait(&B->x_full, 0, 1000000000ull);
-      if (j > 0) mbar_wait(&B->c_full, (j - 1) & 1, 1000000000ull);
+      // drain: wait for the last issued copies of each ring slot
+      if (*reinterpret_cast<volatile int32_t *>(&B->abort_flag)) {
+        for (uint32_t k = nu >= 2 ? nu - 2 : 0; k < nu; ++k)
+          mbar_wait(&B->x_full[k & 1], (k >> 1) & 1, 1000000000ull);
+        for (uint32_t k = gc >= 2 ? gc - 2 : 0; k < gc; ++k) {
+          mbar_wait(&B->c_full[k & 1], (k >> 1) & 1, 1000000000ull);
+          mbar_wait(&B->n_full[k & 1], (k >> 1) & 1, 1000000000ull);
+        }
+      }
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t xb = smem_u32(sX), hb = smem_u32(sHi), lb = smem_u32(sLo);
-      if (km_wait(B, &B->x_full, 0, wait_ns, SITE_KMEANS_MMA)) {
-        for (int j = 0; j < nchunks; ++j) {
-          const int ab = j & 1;
-          if (!km_wait(B, &B->c_full, j & 1, wait_ns, SITE_KMEANS_MMA)) break;
-          if (j >= 2 && !km_wait(B, &B->acc_empty[ab], ((j >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA))
+      uint32_t nu = 0, gc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += grid, ++nu) {
+        const int xs = nu & 1;
+        if (!km_wait(B, &B->x_full[xs], (nu >> 1) & 1, wait_ns, SITE_KMEANS_MMA)) break;
+        const uint32_t xb = smem_u32(smem + Cfg::OFF_X + xs * Cfg::X_BYTES);
+        for (int j = 0; j < nchunks; ++j, ++gc) {
+          const int cs = gc & 1, ab = gc & 1;
+          if (!km_wait(B, &B->c_full[cs], (gc >> 1) & 1, wait_ns, SITE_KMEANS_MMA) ||
+              (gc >= 2 && !km_wait(B, &B->acc_empty[ab], ((gc >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA))) {
+            ok = false;
             break;
+          }
           tc_fence_after();
+          const uint32_t cb = smem_u32(smem + Cfg::OFF_C + cs * 2 * Cfg::C_BYTES);
 #pragma unroll
           for (int part = 0; part < 2; ++part) {
-            const uint32_t cb = part == 0 ? hb : lb;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t koff = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
               mma_bf16_ss(tmem + ab * Cfg::NC, smem_desc_sw128(xb + koff, 16, 1024),
-                          smem_desc_sw128(cb + koff, 16, 1024), Cfg::IDESC,
+                          smem_desc_sw128(cb + part * Cfg::C_BYTES + koff, 16, 1024), Cfg::IDESC,
                           (part == 0 && kk == 0) ? 0u : 1u);
             }
           }
-          mma_commit(&B->c_empty);
+          mma_commit(&B->c_empty[cs]);
           mma_commit(&B->acc_full[ab]);
         }
+        if (ok) mma_commit(&B->x_empty[xs]);   // the unit's MMAs are the last readers of x
       }
       mma_commit(&B->drain);
       mbar_wait(&B->drain, 0, 1000000000ull);
     }
   } else {
-    // epilogue: running best and runner-up over the chunks for token n0 + row
-    const int row = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const float *nh = norms + static_cast<size_t>(h) * Cpad;
-    float best = INFINITY, second = INFINITY;
-    int arg = 0, arg2 = -1;
-    bool ok = true;
-    for (int j = 0; j < nchunks; ++j) {
-      const int ab = j & 1;
-      const bool got = mbar_wait(&B->acc_full[ab], (j >> 1) & 1, wait_ns);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) {
-          record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
-          atomicExch(&B->abort_flag, 1);
+    // ------------------------------------------------------------ epilogue
+    // Two groups of four warps; group g reads accumulator buffer g, i.e. the
+    // chunks with (global chunk index & 1) == g.  Thread `row` of a group =
+    // token n0 + row = TMEM lane row.  Each group keeps the best and runner-up
+    // centroid of its chunks; when a unit has several chunks, group 1 hands
+    // its pair to group 0 through shared memory and group 0 merges.
+    // Near-tie rule: the tensor-core scores carry at most about
+    // 2^-15 ||x|| ||mu|| of error (bf16 split residual plus fp32
+    // accumulation); a runner-up within 2^-14 (||x||^2 + ||mu||^2)
+    // >= 2^-13 ||x|| ||mu|| of the best lists the token for an exact re-check.
+    const int grp = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t nu = 0, gc = 0;
+    for (int u = blockIdx.x; u < units; u += grid, ++nu) {
+      const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
+      const bool valid = n0 + row < N;
+      float best = INFINITY, second = INFINITY;
+      int arg = 0x7fffffff, arg2 = -1;
+      bool ok = true, mine_any = false;
+      for (int j = 0; j < nchunks; ++j, ++gc) {
+        const int ab = gc & 1;
+        if (ab != grp) continue;
+        mine_any = true;
+        const bool got = mbar_wait(&B->acc_full[ab], (gc >> 1) & 1, wait_ns) &&
+                         mbar_wait(&B->n_full[ab], (gc >> 1) & 1, wait_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) {
+            record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
+            atomicExch(&B->abort_flag, 1);
+          }
+          ok = false;
+          break;
         }
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float acc[128];
-      tmem_ld128_sync(tmem + lane_off + ab * Cfg::NC, acc);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B->acc_empty[ab]);
-      const float *cn = nh + j * Cfg::NC;
+        tc_fence_after();
+        float acc[128];
+        tmem_ld128_sync(tmem + lane_off + ab * Cfg::NC, acc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->acc_empty[ab]);
+        const float4 *nv4 = reinterpret_cast<const float4 *>(sNorm + ab * Cfg::NC);
 #pragma unroll
-      for (int c = 0; c < Cfg::NC; ++c) {
-        const float score = fmaf(-2.f, acc[c], __ldg(cn + c));
-        if (score < best) {
-          second = best;
-          arg2 = arg;
-          best = score;
-          arg = j * Cfg::NC + c;
-        } else if (score < second) {
-          second = score;
-          arg2 = j * Cfg::NC + c;
-        }
-      }
-    }
-    if (ok && n0 + row < N) {
-      // Near-tie: the tensor-core scores carry about 2^-15 ||x|| ||mu|| of
-      // error (bf16 split residual plus fp32 accumulation).  When the runner-up
-      // is within 2^-13 (||x||^2 + ||mu||^2) >= 2^-12 ||x|| ||mu||, decide with
-      // the exact float32 distances sum_d (x_d - mu_d)^2 instead.
-      float xr[D];
-#pragma unroll
-      for (int dh = 0; dh < Cfg::DH; ++dh)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(
-              sX + dh * Cfg::HALF + row * 128 + ((q ^ (row & 7)) << 4));
-          const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        for (int c4 = 0; c4 < Cfg::NC / 4; ++c4) {
+          const float4 nv = nv4[c4];
+          const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(b2[e]);
-            xr[dh * 64 + q * 8 + 2 * e] = f.x;
-            xr[dh * 64 + q * 8 + 2 * e + 1] = f.y;
+            const float score = fmaf(-2.f, acc[4 * c4 + e], nn[e]);
+            const int col = j * Cfg::NC + 4 * c4 + e;
+            const bool lt1 = score < best, lt2 = score < second;
+            second = lt1 ? best : (lt2 ? score : second);
+            arg2 = lt1 ? arg : (lt2 ? col : arg2);
+            best = lt1 ? score : best;
+            arg = lt1 ? col : arg;
           }
         }
-      float xx = 0.f;
-#pragma unroll
-      for (int d = 0; d < D; ++d) xx = fmaf(xr[d], xr[d], xx);
-      if (arg2 >= 0 && arg2 < C && second - best <= 0x1p-13f * (xx + __ldg(nh + arg))) {
-        const float *m1 = mu + (static_cast<size_t>(h) * C + arg) * D;
-        const float *m2 = mu + (static_cast<size_t>(h) * C + arg2) * D;
-        float d1 = 0.f, d2 = 0.f;
-#pragma unroll
-        for (int d = 0; d < D; ++d) {
-          const float a1 = xr[d] - __ldg(m1 + d), a2 = xr[d] - __ldg(m2 + d);
-          d1 = fmaf(a1, a1, d1);
-          d2 = fmaf(a2, a2, d2);
-        }
-        if (d2 < d1 || (d2 == d1 && arg2 < arg)) arg = arg2;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->n_empty[ab]);
       }
-      assign[static_cast<size_t>(h) * N + n0 + row] = arg;
+      if (!__all_sync(0xffffffffu, ok)) break;
+      // combine the two groups' pairs when both saw chunks of this unit
+      bool owner = mine_any;
+      if (nchunks >= 2) {
+        const int ms = nu & 1;
+        float4 *slot = sMerge + ms * 128 + row;
+        if (grp == 1) {
+          if (nu >= 2 && !__all_sync(0xffffffffu, mbar_wait(&B->merge_empty[ms], ((nu >> 1) - 1) & 1, wait_ns))) {
+            if (lane == 0) {
+              record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
+              atomicExch(&B->abort_flag, 1);
+            }
+            break;
+          }
+          *slot = make_float4(best, __int_as_float(arg), second, __int_as_float(arg2));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B->merge_full[ms]);
+          owner = false;
+        } else {
+          if (!__all_sync(0xffffffffu, mbar_wait(&B->merge_full[ms], (nu >> 1) & 1, wait_ns))) {
+            if (lane == 0) {
+              record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
+              atomicExch(&B->abort_flag, 1);
+            }
+            break;
+          }
+          const float4 o = *slot;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B->merge_empty[ms]);
+          const float ob = o.x, os = o.z;
+          const int oa = __float_as_int(o.y), oa2 = __float_as_int(o.w);
+          // top two (score, index) of the union of the two pairs
+          if (ob < best || (ob == best && oa < arg)) {
+            if (best < os || (best == os && arg < oa2)) {
+              second = best;
+              arg2 = arg;
+            } else {
+              second = os;
+              arg2 = oa2;
+            }
+            best = ob;
+            arg = oa;
+          } else if (ob < second || (ob == second && oa < arg2)) {
+            second = ob;
+            arg2 = oa;
+          }
+          owner = true;
+        }
+      }
+      if (!owner) continue;
+      const float *nh = norms + static_cast<size_t>(h) * Cpad;
+      const float xx = valid ? __ldg(xnorm + static_cast<size_t>(h) * N + n0 + row) : 0.f;
+      const bool tie = valid && arg2 >= 0 && arg2 < C &&
+                       second - best <= 0x1p-14f * (xx + __ldg(nh + arg));
+      const unsigned tmask = __ballot_sync(0xffffffffu, tie);
+      if (tmask) {   // warp-aggregated append to the near-tie list
+        int base = 0;
+        if (lane == 0) base = atomicAdd(num_ties, __popc(tmask));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (tie) {
+          const int slot = base + __popc(tmask & ((1u << lane) - 1u));
+          ties[slot] = KmTie{h * N + n0 + row, arg, arg2, 0};
+        }
+      }
+      if (valid) assign[static_cast<size_t>(h) * N + n0 + row] = arg;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TM_COLS);
+  }
+}
+
+// ||x_n||^2 in fp32 for every token (x does not change across rounds).
+template <int D>
+__global__ void __launch_bounds__(256) kmeans_xnorm_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                           size_t tokens, float *__restrict__ xnorm) {
+  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= tokens) return;
+  const uint4 *row = reinterpret_cast<const uint4 *>(x + t * D);
+  float s = 0.f;
+#pragma unroll
+  for (int v = 0; v < D / 8; ++v) {
+    const uint4 u = row[v];
+    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(b2[e]);
+      s = fmaf(f.x, f.x, s);
+      s = fmaf(f.y, f.y, s);
+    }
+  }
+  xnorm[t] = s;
+}
+
+// Decides every listed near tie with the exact float32 distances
+// sum_d (x_d - mu_d)^2 (ties to the lower index); one warp per token.
+template <int D>
+__global__ void __launch_bounds__(256) kmeans_refine_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                            int N, int C, const float *__restrict__ mu,
+                                                            const KmTie *__restrict__ ties,
+                                                            const int32_t *__restrict__ num_ties,
+                                                            int32_t *__restrict__ assign) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int nt = *num_ties;
+  for (int e = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); e < nt;
+       e += gridDim.x * (blockDim.x / 32)) {
+    const KmTie t = ties[e];
+    const int h = t.token / N;
+    const __nv_bfloat16 *xr = x + static_cast<size_t>(t.token) * D + lane * PER;
+    const float *m1 = mu + (static_cast<size_t>(h) * C + t.a) * D + lane * PER;
+    const float *m2 = mu + (static_cast<size_t>(h) * C + t.b) * D + lane * PER;
+    float d1 = 0.f, d2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const float xv = __bfloat162float(xr[k]);
+      const float a1 = xv - m1[k], a2 = xv - m2[k];
+      d1 = fmaf(a1, a1, d1);
+      d2 = fmaf(a2, a2, d2);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+      d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+    }
+    if (lane == 0) assign[t.token] = (d2 < d1 || (d2 == d1 && t.b < t.a)) ? t.b : t.a;
   }
 }
 

@@ -20,6 +20,7 @@ namespace {
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 uint64_t g_wait_ns = kDefaultWaitNs;
+int g_fault = 0;
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -95,16 +96,21 @@ struct Carve {
 inline int kmeans_cpad(int C) { return (C + KmCfg<128>::NC - 1) / KmCfg<128>::NC * KmCfg<128>::NC; }
 
 struct KmeansWs {
-  double *sums;
-  float *norms;
+  double *partial;
+  float *norms, *xnorm;
   __nv_bfloat16 *hi, *lo;
-  int32_t *perm, *offsets, *chunk;
+  KmTie *ties;
+  int32_t *perm, *offsets, *chunk, *row_chunks, *num_ties;
 };
 KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
   Carve c{static_cast<uint8_t *>(ws)};
   KmeansWs w;
   const size_t cp = static_cast<size_t>(BH) * kmeans_cpad(C);
-  w.sums = c.take<double>(static_cast<size_t>(BH) * C * D);
+  w.partial = c.take<double>(static_cast<size_t>(BH) * max_accum_chunks(N, C) * D);
+  w.row_chunks = c.take<int32_t>(static_cast<size_t>(BH) * (C + 1));
+  w.xnorm = c.take<float>(static_cast<size_t>(BH) * N);
+  w.ties = c.take<KmTie>(static_cast<size_t>(BH) * N);
+  w.num_ties = c.take<int32_t>(1);
   w.norms = c.take<float>(cp);
   w.hi = c.take<__nv_bfloat16>(cp * D);
   w.lo = c.take<__nv_bfloat16>(cp * D);
@@ -136,10 +142,10 @@ bool sizes_ok(int BH, int N) {
 
 // Stable counting sort of assign[BH,N] by cluster: perm, offsets (and counts).
 svg_status run_sort(const int32_t *assign, int BH, int N, int C, int32_t *perm, int32_t *offsets,
-                    int32_t *counts, int32_t *chunk, cudaStream_t s) {
+                    int32_t *counts, int32_t *chunk, cudaStream_t s, int32_t *row_chunks = nullptr) {
   const int nch = num_chunks(N);
   sort_hist_kernel<<<dim3(nch, BH), 256, 0, s>>>(assign, N, C, chunk);
-  sort_scan_kernel<<<BH, 1024, 0, s>>>(chunk, N, C, nch, offsets, counts);
+  sort_scan_kernel<<<BH, 1024, 0, s>>>(chunk, N, C, nch, offsets, counts, row_chunks, kAccumRows);
   sort_scatter_kernel<<<dim3(nch, BH), 32, 0, s>>>(assign, N, C, chunk, perm);
   return launch_status();
 }
@@ -188,6 +194,8 @@ const char *svg_version(void) { return "svg-b200 0.1 (sm_100a)"; }
 
 void svg_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
 
+void svg_debug_set_fault(int fault) { g_fault = fault; }
+
 svg_status svg_get_error(svg_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return SVG_ERR_CUDA;
@@ -226,11 +234,17 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
       !make_map_bf16(&mlo, w.lo, static_cast<uint64_t>(BH) * Cpad, D, 128))
     return SVG_ERR_CUDA;
   kmeans_split_kernel<<<dim3((Cpad + 7) / 8, BH), 256, 0, s>>>(centroids, C, Cpad, D, w.hi, w.lo,
-                                                              w.norms, w.sums);
-  const dim3 ga((N + 127) / 128, BH);
+                                                              w.norms, w.num_ties);
+  const size_t tokens = static_cast<size_t>(BH) * N;
+  const unsigned xnb = static_cast<unsigned>((tokens + 255) / 256);
+  if (D == 128)
+    kmeans_xnorm_kernel<128><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
+  else
+    kmeans_xnorm_kernel<64><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
+  const int units = BH * ((N + 127) / 128);
+  const int ga = units < num_sms() ? units : num_sms();
   const dim3 gu((C + 7) / 8, BH);
-  const int segs = (N + kAccumRowsPerWarp - 1) / kAccumRowsPerWarp;
-  const dim3 gacc((segs + 7) / 8, BH);
+  const dim3 gacc((max_accum_chunks(N, C) + 7) / 8, BH);
   if (D == 128) {
     if (!set_smem(kmeans_assign_tc_kernel<128>, KmCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
   } else {
@@ -239,20 +253,28 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   for (int it = 0; it < iters; ++it) {
     if (D == 128)
       kmeans_assign_tc_kernel<128><<<ga, KmCfg<128>::THREADS, KmCfg<128>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, N, C, Cpad, w.norms, centroids, assign, g_wait_ns);
+          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
     else
       kmeans_assign_tc_kernel<64><<<ga, KmCfg<64>::THREADS, KmCfg<64>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, N, C, Cpad, w.norms, centroids, assign, g_wait_ns);
-    svg_status st = run_sort(assign, BH, N, C, w.perm, w.offsets, counts, w.chunk, s);
+          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
+    if (D == 128)
+      kmeans_refine_kernel<128><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
+                                                              w.num_ties, assign);
+    else
+      kmeans_refine_kernel<64><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
+                                                             w.num_ties, assign);
+    svg_status st = run_sort(assign, BH, N, C, w.perm, w.offsets, counts, w.chunk, s, w.row_chunks);
     if (st != SVG_OK) return st;
     if (D == 128) {
-      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, assign, w.sums);
-      kmeans_finalize_kernel<128><<<gu, 256, 0, s>>>(C, Cpad, w.offsets, w.sums, centroids, w.hi,
-                                                     w.lo, w.norms);
+      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, w.offsets, w.row_chunks,
+                                                    w.partial);
+      kmeans_finalize_kernel<128><<<gu, 256, 0, s>>>(N, C, Cpad, w.offsets, w.row_chunks, w.partial,
+                                                     centroids, w.hi, w.lo, w.norms, w.num_ties);
     } else {
-      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, assign, w.sums);
-      kmeans_finalize_kernel<64><<<gu, 256, 0, s>>>(C, Cpad, w.offsets, w.sums, centroids, w.hi,
-                                                    w.lo, w.norms);
+      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, w.offsets, w.row_chunks,
+                                                   w.partial);
+      kmeans_finalize_kernel<64><<<gu, 256, 0, s>>>(N, C, Cpad, w.offsets, w.row_chunks, w.partial,
+                                                    centroids, w.hi, w.lo, w.norms, w.num_ties);
     }
   }
   return launch_status();
@@ -378,6 +400,7 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
   prm.BH = BH;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_ns = g_wait_ns;
+  prm.fault = g_fault;
   const int grid = num_sms();
   if (D == 128) {
     using Cfg = AttnCfg<128>;
