@@ -574,55 +574,77 @@ __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
   ktiles[idx] = (slots + 15) >> 4;
 }
 
-// Single block: exclusive scan of q-tile counts, then one AttnItem per q-tile.
+// Single block: one AttnItem per q-tile, ordered for the persistent kernel.
+// Items are sorted by key-tile count, longest first (a counting sort over
+// kAttnBuckets buckets), and the sorted list is laid out in "snake" order:
+// rank r goes to round k = r / grid, slot j = r % grid, reversed on odd
+// rounds.  The attention kernel gives CTA b the items b, b + grid, ..., so
+// every CTA gets one item of each round and the rounds alternate direction,
+// which evens out the work per SM (longest-processing-time-first).
+constexpr int kAttnBuckets = 1024;
+
 __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
     const int32_t *__restrict__ q_off, const int32_t *__restrict__ qtiles,
-    const int32_t *__restrict__ ktiles, int BH, int Cq, AttnItem *__restrict__ items,
+    const int32_t *__restrict__ ktiles, int BH, int Cq, int grid, AttnItem *__restrict__ items,
     int32_t *__restrict__ num_items) {
+  __shared__ int hist[kAttnBuckets];
   __shared__ int warp_tot[32];
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
   const int total = BH * Cq;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  for (int base = 0; base < total; base += 1024) {
-    const int idx = base + threadIdx.x;
-    const int v = idx < total ? qtiles[idx] : 0;
-    int incl = v;
+  hist[threadIdx.x] = 0;
+  __syncthreads();
+  // bucket b = kAttnBuckets - 1 - min(kt, kAttnBuckets - 1): descending cost
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int v = qtiles[idx];
+    if (v > 0) atomicAdd(&hist[kAttnBuckets - 1 - min(ktiles[idx], kAttnBuckets - 1)], v);
+  }
+  __syncthreads();
+  // exclusive scan of the buckets (one per thread)
+  const int v = hist[threadIdx.x];
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int t = warp_tot[lane];
+    int ti = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
     }
-    if (lane == 31) warp_tot[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      const int t = warp_tot[lane];
-      int ti = t;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, ti, o);
-        if (lane >= o) ti += y;
-      }
-      warp_tot[lane] = ti - t;
-    }
-    __syncthreads();
-    const int start = carry + warp_tot[w] + incl - v;
-    if (idx < total && v > 0) {
-      const int h = idx / Cq, i = idx % Cq;
-      const int r0 = q_off[h * (Cq + 1) + i], r1 = q_off[h * (Cq + 1) + i + 1];
-      const int kt = ktiles[idx];
-      for (int t = 0; t < v; ++t) {
-        const int q0 = r0 + t * 128;
-        const int rows = min(128, r1 - q0);
-        items[start + t] = AttnItem{h, i, q0, rows | (kt << 8)};
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == 1023) carry = start + v;
-    __syncthreads();
+    warp_tot[lane] = ti - t;
   }
-  if (threadIdx.x == 0) *num_items = carry;
+  __syncthreads();
+  const int excl = warp_tot[w] + incl - v;
+  __syncthreads();
+  hist[threadIdx.x] = excl;                       // now: next free rank of each bucket
+  if (threadIdx.x == kAttnBuckets - 1) {
+    *num_items = excl + v;
+    warp_tot[0] = excl + v;
+  }
+  __syncthreads();
+  const int n_items = warp_tot[0];
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int qt = qtiles[idx];
+    if (qt <= 0) continue;
+    const int kt = ktiles[idx];
+    const int r0 = atomicAdd(&hist[kAttnBuckets - 1 - min(kt, kAttnBuckets - 1)], qt);
+    const int h = idx / Cq, i = idx % Cq;
+    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_off[h * (Cq + 1) + i + 1];
+    for (int t = 0; t < qt; ++t) {
+      const int rank = r0 + t;
+      const int round = rank / grid, slot = rank % grid;
+      const int in_round = min(grid, n_items - round * grid);   // the last round may be partial
+      const int pos = round * grid + ((round & 1) ? in_round - 1 - slot : slot);
+      const int q0 = row0 + t * 128;
+      items[pos] = AttnItem{h, i, q0, min(128, row1 - q0) | (kt << 8)};
+    }
+  }
 }
 
 }  // namespace svg

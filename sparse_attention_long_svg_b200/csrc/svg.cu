@@ -373,8 +373,8 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
   const int pairs = BH * Cq;
   attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
                                                             Cq, Ck, w.qtiles, w.ktiles);
-  attn_plan_emit_kernel<<<1, 1024, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, w.items,
-                                           w.num_items);
+  attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, num_sms(),
+                                                   w.items, w.num_items);
   svg_status st = launch_status();
   if (st != SVG_OK) return st;
 
