@@ -100,7 +100,7 @@ class ClockSampler:
         try:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -296,6 +296,9 @@ def run_svg(args, wl):
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    svg.profile_enable(True)             # live per-kernel CUDA-event timing of the two heavy kernels
+    svg.profile_read("kmeans_assign")
+    svg.profile_read("sparse_attn")
     if True:
         t_start.record()
         for s in range(args.steps):
@@ -303,6 +306,9 @@ def run_svg(args, wl):
         t_end.record()
         torch.cuda.synchronize()
     clocks.__exit__(None, None, None)
+    assign_ms, assign_n, _ = svg.profile_read("kmeans_assign")
+    attn_k_ms, attn_n, _ = svg.profile_read("sparse_attn")
+    svg.profile_enable(False)
     if world > 1:
         torch.distributed.barrier()
     local_ms = t_start.elapsed_time(t_end)
@@ -347,15 +353,32 @@ def run_svg(args, wl):
     h2d = int(3 * hq.numel() * 2 + 2 * hmq.numel() * 4)
     d2h = int(hout.numel() * 2)
 
-    # ---- rooflines
+    # ---- rooflines of the two heavy kernels, from the live event timings
     tc_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     attn_tflops = flops_layer / (stage_ms["attn"] * 1e-3) / 1e12
-    traffic = load_traffic("sparse_attn_kernel", wl.name)
-    roofline = {"kernel": f"sparse_attn_kernel<{D}>", "bound": "tensor", "achieved": attn_tflops,
-                "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_tflops / tc_peak, "traffic": traffic,
-                "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a multi-ms step)",
-                "algorithmic": "4*D*sum_selected(n_q*n_k) FLOP per launch = %.4g" % flops_layer}
+    peak_note = f"{peak_kind} bf16 sustained (kernel timed inside a multi-ms step)"
+    attn_kernel_ms = attn_k_ms / max(attn_n, 1)
+    attn_kernel_tflops = flops_layer / (attn_kernel_ms * 1e-3) / 1e12
+    roof_attn = {"kernel": f"sparse_attn_kernel<{D}>", "bound": "tensor", "achieved": attn_kernel_tflops,
+                 "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_kernel_tflops / tc_peak,
+                 "traffic": load_traffic("sparse_attn_kernel", wl.name), "peak_kind": peak_note,
+                 "launch_ms": attn_kernel_ms, "launches": attn_n, "total_ms": attn_k_ms,
+                 "algorithmic": "4*D*sum_selected(n_q*n_k) = %.4g FLOP per launch" % flops_layer}
+    # assign launches alternate: iters on Q (C = cq) then iters on K (C = ck) per step
+    assign_flops = 2.0 * N * D * BH * wl.iters * (wl.cq + wl.ck) * args.steps
+    assign_launch_ms = assign_ms / max(assign_n, 1)
+    assign_tflops = assign_flops / (assign_ms * 1e-3) / 1e12 if assign_ms > 0 else 0.0
+    roof_assign = {"kernel": f"kmeans_assign_tc_kernel<{D}>", "bound": "tensor", "achieved": assign_tflops,
+                   "peak": tc_peak, "unit": "TFLOP/s", "frac": assign_tflops / tc_peak,
+                   "traffic": load_traffic("kmeans_assign_tc_kernel", wl.name), "peak_kind": peak_note,
+                   "launch_ms": assign_launch_ms, "launches": assign_n, "total_ms": assign_ms,
+                   "algorithmic": "2*N*C*D*BH FLOP per launch (distance contraction; C = %d or %d)"
+                                  % (wl.cq, wl.ck)}
+    if assign_ms > attn_k_ms:
+        roofline, roofline_other = roof_assign, roof_attn
+    else:
+        roofline, roofline_other = roof_attn, roof_assign
     tensor_bytes = BH * N * D * 2
     km_flops = {c: 2.0 * N * c * D * BH * wl.iters for c in (wl.cq, wl.ck)}
     km_bytes = 2.0 * tensor_bytes * wl.iters          # assign read + update read per round
@@ -391,7 +414,7 @@ def run_svg(args, wl):
             "config": workload_config(wl, world),
             "attn_ms": stage_ms["attn"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
-            "roofline": roofline, "cpu_baseline": cpu,
+            "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": kernel_launches_per_step(wl) * args.steps,

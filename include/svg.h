@@ -202,6 +202,20 @@ void svg_set_wait_timeout_ns(uint64_t ns);
  * restores normal operation.  Outputs of a faulted launch are undefined. */
 void svg_debug_set_fault(int fault);
 
+/* ------------------------------------------------------------------------ kernel timing
+ * Live per-kernel timing for benchmarks.  While enabled, the library records
+ * a pair of CUDA events on the caller's stream around every launch of its two
+ * heavy kernels: kernel 0 = the k-means assign kernel (inside svg_kmeans),
+ * kernel 1 = the block-sparse attention kernel (inside svg_sparse_attn,
+ * without its planning kernels).  Events come from a fixed pool created on
+ * the first enable (up to 1024 launches between reads; later launches are not
+ * timed and are reported in `dropped`).  svg_profile_read waits for the
+ * recorded events, returns the summed milliseconds and the number of timed
+ * launches of one kernel since the previous read, and resets that kernel's
+ * record.  Timing adds two event records per launch and nothing else. */
+svg_status svg_profile_enable(int on);
+svg_status svg_profile_read(int kernel, double *ms, int *launches, int *dropped);
+
 /* Library version, e.g. "svg-b200 0.1 (sm_100a)". */
 const char *svg_version(void);
 

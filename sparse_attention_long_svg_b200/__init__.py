@@ -46,7 +46,12 @@ SIGNATURES = {
     "svg_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "svg_sparse_attn_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P]),
+    "svg_profile_enable": (_I, [_I]),
+    "svg_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
+                              ctypes.POINTER(ctypes.c_int)]),
 }
+
+PROFILE_KERNELS = {"kmeans_assign": 0, "sparse_attn": 1}
 
 NOALLOC_SCRATCH_BYTES = 2 << 20   # SVG_NOALLOC_SCRATCH_BYTES in include/svg.h
 
@@ -112,6 +117,19 @@ def get_error(stream=None) -> int:
 
 def set_wait_timeout_ns(ns: int):
     load_library().svg_set_wait_timeout_ns(int(ns))
+
+
+def profile_enable(on: bool = True):
+    """Live timing of the k-means assign and attention kernels (see svg_profile_enable)."""
+    _check("svg_profile_enable", load_library().svg_profile_enable(1 if on else 0))
+
+
+def profile_read(kernel: str) -> Tuple[float, int, int]:
+    """(summed ms, timed launches, untimed launches) of a kernel since the last read."""
+    ms, n, dropped = ctypes.c_double(), ctypes.c_int(), ctypes.c_int()
+    _check("svg_profile_read", load_library().svg_profile_read(PROFILE_KERNELS[kernel], ctypes.byref(ms),
+                                                               ctypes.byref(n), ctypes.byref(dropped)))
+    return ms.value, n.value, dropped.value
 
 
 # --------------------------------------------------------------------- stages

@@ -345,10 +345,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       while (wp < total) {
         bool progress = false;
         if (ws < total && gs < gp + 2) {
-          if (!q_ok) q_ok = mbar_try_wait(&B->q_full, n_s & 1);
+          if (!q_ok) q_ok = mbar_test(&B->q_full, n_s & 1);
           const int st = gs & 1;
-          if (q_ok && mbar_try_wait(&B->k_full[st], (gs >> 1) & 1) &&
-              (gs < 2 || mbar_try_wait(&B->s_free[st], ((gs >> 1) - 1) & 1))) {
+          if (q_ok && mbar_test(&B->k_full[st], (gs >> 1) & 1) &&
+              (gs < 2 || mbar_test(&B->s_free[st], ((gs >> 1) - 1) & 1))) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
         if (gp < gs) {
           const int vs = static_cast<int>(gp % 3);
-          if (mbar_try_wait(&B->p_full, gp & 1) && mbar_try_wait(&B->v_full[vs], (gp / 3) & 1)) {
+          if (mbar_test(&B->p_full, gp & 1) && mbar_test(&B->v_full[vs], (gp / 3) & 1)) {
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < Cfg::BN / 16; ++kk) {

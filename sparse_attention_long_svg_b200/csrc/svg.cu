@@ -173,9 +173,65 @@ svg_status run_row_move(bool gather, int ntensors, const void *const *src, void 
   return launch_status();
 }
 
+// --------------------------------------------------------------- kernel timing
+// Event pairs recorded around the assign and attention launches while
+// profiling is enabled (see svg_profile_enable in svg.h).
+constexpr int kProfKernels = 2, kProfSlots = 1024;
+struct ProfState {
+  bool on = false, created = false;
+  cudaEvent_t ev[kProfKernels][kProfSlots][2];
+  int used[kProfKernels] = {0, 0};
+  int dropped[kProfKernels] = {0, 0};
+};
+ProfState g_prof;
+std::mutex g_prof_mutex;
+
+// Returns the event pair to record around one launch, or nullptr.
+cudaEvent_t *prof_slot(int kernel) {
+  if (!g_prof.on) return nullptr;
+  std::lock_guard<std::mutex> lock(g_prof_mutex);
+  if (g_prof.used[kernel] >= kProfSlots) {
+    ++g_prof.dropped[kernel];
+    return nullptr;
+  }
+  return g_prof.ev[kernel][g_prof.used[kernel]++];
+}
+
 }  // namespace
 
 extern "C" {
+
+svg_status svg_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_prof_mutex);
+  if (on && !g_prof.created) {
+    for (int k = 0; k < kProfKernels; ++k)
+      for (int i = 0; i < kProfSlots; ++i)
+        for (int j = 0; j < 2; ++j)
+          if (cudaEventCreate(&g_prof.ev[k][i][j]) != cudaSuccess) return SVG_ERR_CUDA;
+    g_prof.created = true;
+  }
+  g_prof.on = on != 0;
+  return SVG_OK;
+}
+
+svg_status svg_profile_read(int kernel, double *ms, int *launches, int *dropped) {
+  if (kernel < 0 || kernel >= kProfKernels || !ms || !launches) return SVG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_prof_mutex);
+  double total = 0.0;
+  for (int i = 0; i < g_prof.used[kernel]; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[kernel][i][1]) != cudaSuccess) return SVG_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, g_prof.ev[kernel][i][0], g_prof.ev[kernel][i][1]) != cudaSuccess)
+      return SVG_ERR_CUDA;
+    total += t;
+  }
+  *ms = total;
+  *launches = g_prof.used[kernel];
+  if (dropped) *dropped = g_prof.dropped[kernel];
+  g_prof.used[kernel] = 0;
+  g_prof.dropped[kernel] = 0;
+  return SVG_OK;
+}
 
 const char *svg_status_string(svg_status s) {
   switch (s) {
@@ -251,12 +307,15 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
     if (!set_smem(kmeans_assign_tc_kernel<64>, KmCfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
   }
   for (int it = 0; it < iters; ++it) {
+    cudaEvent_t *pe = prof_slot(0);
+    if (pe) cudaEventRecord(pe[0], s);
     if (D == 128)
       kmeans_assign_tc_kernel<128><<<ga, KmCfg<128>::THREADS, KmCfg<128>::SMEM_BYTES, s>>>(
           mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
     else
       kmeans_assign_tc_kernel<64><<<ga, KmCfg<64>::THREADS, KmCfg<64>::SMEM_BYTES, s>>>(
           mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
+    if (pe) cudaEventRecord(pe[1], s);
     if (D == 128)
       kmeans_refine_kernel<128><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
                                                               w.num_ties, assign);
@@ -402,6 +461,8 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
   prm.wait_ns = g_wait_ns;
   prm.fault = g_fault;
   const int grid = num_sms();
+  cudaEvent_t *pe = prof_slot(1);
+  if (pe) cudaEventRecord(pe[0], s);
   if (D == 128) {
     using Cfg = AttnCfg<128>;
     if (!set_smem(sparse_attn_kernel<128>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
@@ -411,6 +472,7 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
     if (!set_smem(sparse_attn_kernel<64>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
     sparse_attn_kernel<64><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
   }
+  if (pe) cudaEventRecord(pe[1], s);
   return launch_status();
 }
 
