@@ -158,9 +158,9 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
  * every GPU which loads the library holds until the process exits.
  *
  *  - Limit: svg_sparse_attn_workspace_size(BH, N, Cq), about
- *    16*BH*(ceil(N/128) + Cq) + 8*BH*Cq bytes, must not exceed
+ *    16*BH*(ceil(N/256) + Cq) + 8*BH*Cq bytes, must not exceed
  *    SVG_NOALLOC_SCRATCH_BYTES (e.g. 80 heads x 75,600 tokens x 200 q-clusters
- *    needs 1.2 MB); larger sizes return SVG_ERR_WORKSPACE before anything is
+ *    needs 0.8 MB); larger sizes return SVG_ERR_WORKSPACE before anything is
  *    launched.
  *  - It allocates and frees nothing (no cudaMalloc, no cudaFree, no
  *    allocating library routine).

@@ -5,64 +5,70 @@
 // permuted K/V and are gathered sparsely, without padding them to fixed
 // block sizes).
 //
-// Work unit: 128 consecutive permuted query rows of one q-cluster ("q-tile").
-// Its key list is the concatenation of the selected k-clusters' row ranges,
-// cut into 8-row slots; 16 slots form a 128-key tile.  A k-cluster of n rows
-// costs ceil(n/8) slots and at most 7 masked rows; it is fetched with as few
-// TMA boxes as possible (boxes of 8..128 rows, a power of two that fits the
-// rest of the cluster and the rest of the tile).  Rows past a cluster's end
-// inside its last slot are masked out of the softmax.
+// Work item: up to 256 consecutive permuted query rows of one q-cluster, as
+// two 128-row tiles A and B that share every K/V tile (one K/V fetch feeds
+// two tiles of MMAs).  The item's key list is the concatenation of its
+// selected k-clusters' row ranges (touching ranges merged into runs), cut
+// into 8-row slots; 8 slots form a 64-key tile.  A run of n rows costs
+// ceil(n/8) slots and at most 7 masked rows, fetched with as few TMA boxes as
+// possible (8, 16, 32 or 64 rows: the largest power of two that fits the rest
+// of the run and of the tile).
 //
-// Per CTA (persistent, one per SM), 7 warps:
-//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t)
-//   warp 4     TMA producer: Q tile, K and V boxes into 2- and 3-stage rings
-//   warp 5     MMA issuer: S = Q K^T into TMEM (double-buffered) and
-//              O += P V into TMEM; issues whichever of the two is ready
-//              first; also owns the TMEM allocation
-//   warp 6     item loader: the next q-tile's selected key ranges, read from
-//              global memory into a 2-entry shared-memory ring ahead of time
-// Per key tile k: S(k) -> softmax(k) writes P(k) (bf16 pairs, TMEM) ->
-// PV(k) with A = P read from TMEM.  O accumulates in TMEM across the key
-// tiles of a q-tile; the softmax warps rescale it in place only when a row's
-// running max grows by more than 2^8 (exact: every probability is taken
-// against the same reference max that O and the row sum use).
+// Per CTA (persistent, one per SM), 11 warps:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t owns
+//              query row t of its tile (TMEM lane t)
+//   warp 8     TMA producer: Q tiles, K and V boxes into 3-stage rings
+//   warp 9     MMA issuer: S_x = Q_x K^T into TMEM (two buffers per tile) and
+//              O_x += P_x V into TMEM, issuing whichever is ready; owns TMEM
+//   warp 10    item loader: the next item's key ranges into shared memory
+// P is written by the softmax warps to shared memory (bf16, 128-byte
+// swizzled, K-major) so both MMAs read their operands from shared memory.
+// O accumulates in TMEM across the item's key tiles; the softmax warps
+// rescale it in place only when a row's running max grows by more than 2^8
+// (exact: every probability is taken against the same reference max that O
+// and the row sum use).
 #pragma once
 #include "common.cuh"
 
 namespace svg {
 
-struct AttnItem {  // one q-tile
-  int32_t h, i, q0, packed;  // packed = rows (<=128) | key_tiles << 8
+constexpr int kItemRows = 256;     // query rows per work item (two 128-row tiles)
+constexpr int kSlotsPerTile = 8;   // 8-row slots per 64-key tile
+
+struct AttnItem {  // up to 256 query rows of one q-cluster
+  int32_t h, i, q0, packed;  // packed = rows (<= 256) | key_tiles << 9
 };
 
 template <int D>
 struct AttnCfg {
-  static constexpr int BM = 128, BN = 128, SLOT = 8, NSLOT = BN / SLOT;
+  static constexpr int BM = 128, BN = 64, SLOT = 8, NSLOT = BN / SLOT;
   static constexpr int DH = D / 64;  // 64-channel (128-byte) halves
-  static constexpr int KST = 2;      // K ring depth
-  static constexpr int VST = 3;      // V ring depth (V(t) is issued only once PV(t - VST) is done)
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int HALF_Q = BM * 128;   // bytes of one 64-channel half of Q
-  static constexpr int HALF_KV = BN * 128;  // same for a K/V tile
+  static constexpr int KST = 3, VST = 3;
+  static constexpr int QT_BYTES = BM * D * 2;   // one Q tile
+  static constexpr int KV_BYTES = BN * D * 2;   // one K or V tile
+  static constexpr int P_BYTES = BM * BN * 2;   // one P tile
+  static constexpr int HALF_Q = BM * 128;       // one 64-channel half of a Q tile
+  static constexpr int HALF_KV = BN * 128;      // same for a K/V tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int MAX_SEL = 1024;                      // selected k-clusters per q-cluster
-  static constexpr int OFF_RANGES = OFF_V + VST * KV_BYTES; // 2 x int2 (first row, rows) per selection
+  static constexpr int OFF_P = OFF_V + VST * KV_BYTES;
+  static constexpr int MAX_SEL = 1024;                        // selected k-clusters per q-cluster
+  static constexpr int OFF_RANGES = OFF_P + 2 * P_BYTES;      // 2 x int2 (first row, rows)
   static constexpr int OFF_BAR = OFF_RANGES + 2 * MAX_SEL * 8;
-  static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers/meta + alignment slack
-  static constexpr uint32_t TM_S = 0;      // two S buffers: columns [0,128) and [128,256)
-  static constexpr uint32_t TM_O = 256;    // O: columns [256, 256 + D)
-  static constexpr uint32_t TM_P = 384;    // P (bf16 pairs): columns [384, 448)
+  static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;    // barriers/meta + alignment slack
+  // TMEM: S of tile x in buffer b at x*128 + b*64 (64 columns); O of tile x at 256 + x*128
   static constexpr uint32_t TM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
-  static constexpr int THREADS = 224;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, LOADER_WARP = 10;
+  static constexpr int THREADS = 11 * 32;
+  __device__ static constexpr uint32_t tm_s(int x, int b) { return x * 128 + b * 64; }
+  __device__ static constexpr uint32_t tm_o(int x) { return 256 + x * 128; }
 };
 
-// TMA boxes of 8, 16, 32, 64 and 128 rows (one tensor map each for K and V).
-constexpr int kNumBoxSizes = 5;
+// TMA boxes of 8, 16, 32 and 64 rows (one tensor map each for K and V).
+constexpr int kNumBoxSizes = 4;
 
 struct AttnMaps {
   CUtensorMap q;
@@ -70,12 +76,11 @@ struct AttnMaps {
   CUtensorMap v[kNumBoxSizes];
 };
 
-// Sets bits [first, first + count) of a 128-bit mask held in four registers
-// (word-level arithmetic; no per-bit loop, no dynamic indexing).
-__device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count) {
+// Sets bits [first, first + count) of a 64-bit mask held in two registers.
+__device__ __forceinline__ void set_bits(uint32_t (&m)[2], int first, int count) {
   const int last = first + count;
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < 2; ++w) {
     const int lo = max(first, 32 * w), hi = min(last, 32 * w + 32);
     if (hi > lo) {
       const int n = hi - lo;
@@ -87,14 +92,14 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count)
 
 struct AttnBarriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[3], v_empty[3], meta_full[3];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, o_full;
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3], meta_full[3];
+  uint64_t s_full[2][2], s_free[2][2];   // [tile][buffer]
+  uint64_t p_full[2], o_full[2];         // [tile]
   uint64_t item_full[2], item_empty[2];
   uint64_t drain;
   AttnItem item[2];      // item ring written by the loader warp
   int32_t item_cnt[2];
-  uint32_t meta[3][4];   // per V stage: 128-bit key validity mask of the tile
+  uint32_t meta[3][2];   // per V stage: 64-bit key validity mask of the tile
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -108,7 +113,7 @@ struct AttnParams {
   int N, Cq, Ck, BH;
   float scale_log2;      // softmax scale * log2(e)
   uint64_t wait_ns;
-  int fault;             // test hook: 1 = never load the query tile (waits must run out)
+  int fault;             // test hook: 1 = never load the query tiles (waits must run out)
 };
 
 __device__ __forceinline__ bool attn_wait(AttnBarriers *b, uint64_t *bar, uint32_t parity,
@@ -150,6 +155,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint8_t *sQ = smem + Cfg::OFF_Q;
   uint8_t *sK = smem + Cfg::OFF_K;
   uint8_t *sV = smem + Cfg::OFF_V;
+  uint8_t *sP = smem + Cfg::OFF_P;
   int2 *sRanges = reinterpret_cast<int2 *>(smem + Cfg::OFF_RANGES);
   AttnBarriers *B = reinterpret_cast<AttnBarriers *>(smem + Cfg::OFF_BAR);
   const int warp = static_cast<int>(warp_id());
@@ -159,29 +165,31 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     mbar_init(&B->q_full, 1);
     mbar_init(&B->q_empty, 1);
     for (int s = 0; s < 3; ++s) {
+      mbar_init(&B->k_full[s], 1);
+      mbar_init(&B->k_empty[s], 1);
       mbar_init(&B->v_full[s], 1);
       mbar_init(&B->v_empty[s], 1);
       mbar_init(&B->meta_full[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&B->k_full[s], 1);
-      mbar_init(&B->k_empty[s], 1);
-      mbar_init(&B->s_full[s], 1);
-      mbar_init(&B->s_free[s], 4);
-      mbar_init(&B->item_full[s], 1);
-      mbar_init(&B->item_empty[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&B->s_full[x][b], 1);
+        mbar_init(&B->s_free[x][b], 4);
+      }
+      mbar_init(&B->p_full[x], 4);
+      mbar_init(&B->o_full[x], 1);
+      mbar_init(&B->item_full[x], 1);
+      mbar_init(&B->item_empty[x], 1);
     }
-    mbar_init(&B->p_full, 4);
-    mbar_init(&B->o_full, 1);
     mbar_init(&B->drain, 1);
     B->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     tmem_alloc(&B->tmem_base, Cfg::TM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == Cfg::PRODUCER_WARP && lane == 0) {
     tma_prefetch_desc(&maps.q);
     for (int b = 0; b < kNumBoxSizes; ++b) {
       tma_prefetch_desc(&maps.k[b]);
@@ -196,7 +204,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   const uint64_t ns = P.wait_ns;
   const int grid = static_cast<int>(gridDim.x);
 
-  if (warp == 6) {
+  if (warp == Cfg::LOADER_WARP) {
     // ------------------------------------------------------------ item loader
     int n = 0;
     for (int w = blockIdx.x; w < total; w += grid, ++n) {
@@ -219,18 +227,30 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
         dst[c] = r;
       }
-      if (lane == 0) {
+      __syncwarp();
+      if (lane == 0) {   // merge touching ranges into runs (same rule as the planning kernel)
+        int m = 0, run_end = -1;
+        for (int c = 0; c < cnt; ++c) {
+          const int2 r = dst[c];
+          if (r.y <= 0) continue;
+          if (m > 0 && r.x == run_end) {
+            dst[m - 1].y += r.y;
+          } else {
+            dst[m++] = r;
+          }
+          run_end = r.x + r.y;
+        }
         B->item[buf] = it;
-        B->item_cnt[buf] = cnt;
+        B->item_cnt[buf] = m;
       }
       __threadfence_block();
       __syncwarp();
       if (lane == 0) mbar_arrive(&B->item_full[buf]);
     }
-  } else if (warp == 4) {
+  } else if (warp == Cfg::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
-    uint32_t g = 0;            // global key-tile counter
-    uint32_t nq = 0, gk = 0, gv = 0;  // Q tiles, K tiles and V tiles issued (for the drain)
+    uint32_t g = 0;                  // global key-tile counter
+    uint32_t nq = 0, gk = 0, gv = 0;  // Q loads, K tiles and V tiles issued (for the drain)
     int n_items = 0;
     if (lane == 0) {
       bool ok = true;
@@ -240,28 +260,32 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const AttnItem it = B->item[buf];
         const int cnt = B->item_cnt[buf];
         const int2 *ranges = sRanges + buf * Cfg::MAX_SEL;
-        const int ntk = it.packed >> 8;
+        const int ntk = it.packed >> 9;
+        const bool has_b = (it.packed & 0x1FF) > Cfg::BM;
         if (n_items > 0 && !attn_wait(B, &B->q_empty, (n_items - 1) & 1, ns, SITE_ATTN_PRODUCER))
           break;
         if (P.fault != 1) {
-          mbar_arrive_expect_tx(&B->q_full, Cfg::Q_BYTES);
+          mbar_arrive_expect_tx(&B->q_full, Cfg::QT_BYTES * (has_b ? 2 : 1));
           const int qrow = it.h * P.N + it.q0;
 #pragma unroll
-          for (int dh = 0; dh < Cfg::DH; ++dh)
-            tma_load_2d(sQ + dh * Cfg::HALF_Q, &maps.q, dh * 64, qrow, &B->q_full);
+          for (int x = 0; x < 2; ++x) {
+            if (x == 1 && !has_b) break;
+#pragma unroll
+            for (int dh = 0; dh < Cfg::DH; ++dh)
+              tma_load_2d(sQ + x * Cfg::QT_BYTES + dh * Cfg::HALF_Q, &maps.q, dh * 64,
+                          qrow + x * Cfg::BM, &B->q_full);
+          }
           ++nq;
         }
         int ci = 0, cur = 0, left = 0;
         const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
         for (int t = 0; t < ntk; ++t, ++g) {
-          const int st = g & 1;
-          const uint32_t ph = (g >> 1) & 1;
-          const int vs = static_cast<int>(g % 3);
-          const uint32_t vph = (g / 3) & 1;
-          // Cut the tile into boxes of 1, 2, 4, 8 or 16 slots (8..128 rows): the
-          // largest power of two that fits both the tile and the cluster rest.
+          const int ks = static_cast<int>(g % 3);
+          const uint32_t kph = (g / 3) & 1;
+          // Cut the tile into boxes of 1, 2, 4 or 8 slots (8..64 rows): the
+          // largest power of two that fits both the tile and the run rest.
           int box_row[Cfg::NSLOT], box_kind[Cfg::NSLOT], nbox = 0;
-          uint32_t mask[4] = {0, 0, 0, 0};
+          uint32_t mask[2] = {0, 0};
           int sl = 0;
           while (sl < Cfg::NSLOT) {
             while (left <= 0 && ci < cnt) {
@@ -286,31 +310,29 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             ++nbox;
             sl += nsl;
           }
-          if (g >= 2 && !attn_wait(B, &B->k_empty[st], ph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
-          mbar_arrive_expect_tx(&B->k_full[st], Cfg::KV_BYTES);
-          uint8_t *kdst = sK + st * Cfg::KV_BYTES;
+          if (g >= 3 && !attn_wait(B, &B->k_empty[ks], kph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(&B->k_full[ks], Cfg::KV_BYTES);
+          uint8_t *kdst = sK + ks * Cfg::KV_BYTES;
           for (int bx = 0; bx < nbox; ++bx) {
             const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
 #pragma unroll
             for (int dh = 0; dh < Cfg::DH; ++dh)
               tma_load_2d(kdst + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64, box_row[bx],
-                          &B->k_full[st]);
+                          &B->k_full[ks]);
           }
           gk = g + 1;
-          if (g >= 3 && !attn_wait(B, &B->v_empty[vs], vph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
-          B->meta[vs][0] = mask[0];
-          B->meta[vs][1] = mask[1];
-          B->meta[vs][2] = mask[2];
-          B->meta[vs][3] = mask[3];
-          mbar_arrive(&B->meta_full[vs]);
-          mbar_arrive_expect_tx(&B->v_full[vs], Cfg::KV_BYTES);
-          uint8_t *vdst = sV + vs * Cfg::KV_BYTES;
+          if (g >= 3 && !attn_wait(B, &B->v_empty[ks], kph ^ 1, ns, SITE_ATTN_PRODUCER)) { ok = false; break; }
+          B->meta[ks][0] = mask[0];
+          B->meta[ks][1] = mask[1];
+          mbar_arrive(&B->meta_full[ks]);
+          mbar_arrive_expect_tx(&B->v_full[ks], Cfg::KV_BYTES);
+          uint8_t *vdst = sV + ks * Cfg::KV_BYTES;
           for (int bx = 0; bx < nbox; ++bx) {
             const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
 #pragma unroll
             for (int dh = 0; dh < Cfg::DH; ++dh)
               tma_load_2d(vdst + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64, box_row[bx],
-                          &B->v_full[vs]);
+                          &B->v_full[ks]);
           }
           gv = g + 1;
         }
@@ -320,80 +342,107 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       // last phase of each so no copy is in flight when the CTA exits.
       if (aborted(B)) {
         if (nq > 0) mbar_wait(&B->q_full, (nq - 1) & 1, 1000000000ull);
-        for (uint32_t k = (gk >= 2 ? gk - 2 : 0); k < gk; ++k)
-          mbar_wait(&B->k_full[k & 1], (k >> 1) & 1, 1000000000ull);
+        for (uint32_t k = (gk >= 3 ? gk - 3 : 0); k < gk; ++k)
+          mbar_wait(&B->k_full[k % 3], (k / 3) & 1, 1000000000ull);
         for (uint32_t k = (gv >= 3 ? gv - 3 : 0); k < gv; ++k)
           mbar_wait(&B->v_full[k % 3], (k / 3) & 1, 1000000000ull);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    // Two cursors walk this CTA's key tiles: gs = next S, gp = next PV.  Each
-    // pass issues whichever is ready (S first), so neither waits behind the
-    // other's operands.  S may run at most two tiles ahead (two S buffers).
+    // Two cursors walk this CTA's key tiles: gs = next tile for S, gp = next
+    // tile for PV; each tile has one S (and one PV) per query tile present.
+    // Every pass issues whatever is ready (S first), so neither waits behind
+    // the other's operands.
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV),
+                     p_base = smem_u32(sP);
       int ws = blockIdx.x, wp = blockIdx.x, n_s = 0;
       int ts = 0, tp = 0;
-      int ntk_s = ws < total ? (P.items[ws].packed >> 8) : 0;
-      int ntk_p = ntk_s;
-      int ntk_next = ws + grid < total ? (P.items[ws + grid].packed >> 8) : 0;
+      int pk_s = ws < total ? P.items[ws].packed : 0;
+      int pk_p = pk_s;
+      int pk_next = ws + grid < total ? P.items[ws + grid].packed : 0;
       uint32_t gs = 0, gp = 0;
+      uint32_t n_sx[2] = {0, 0}, n_px[2] = {0, 0};
+      bool s_done[2] = {false, false}, p_done[2] = {false, false};
       bool q_ok = false;
       const long long limit = static_cast<long long>(ns) * 2;
       long long t_last = clock64();
       while (wp < total) {
         bool progress = false;
-        if (ws < total && gs < gp + 2) {
+        if (ws < total) {
+          const int ks = static_cast<int>(gs % 3);
+          const bool has_b = (pk_s & 0x1FF) > Cfg::BM;
           if (!q_ok) q_ok = mbar_test(&B->q_full, n_s & 1);
-          const int st = gs & 1;
-          if (q_ok && mbar_test(&B->k_full[st], (gs >> 1) & 1) &&
-              (gs < 2 || mbar_test(&B->s_free[st], ((gs >> 1) - 1) & 1))) {
-            tc_fence_after();
+          if (q_ok && mbar_test(&B->k_full[ks], (gs / 3) & 1)) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * Cfg::HALF_Q + (kk & 3) * 32;
-              const uint64_t a = smem_desc_sw128(q_base + koff, 16, 1024);
-              const uint64_t b = smem_desc_sw128(
-                  k_base + st * Cfg::KV_BYTES + (kk >> 2) * Cfg::HALF_KV + (kk & 3) * 32, 16, 1024);
-              mma_bf16_ss(tmem + Cfg::TM_S + st * 128, a, b, Cfg::IDESC_S, kk > 0 ? 1u : 0u);
+            for (int x = 0; x < 2; ++x) {
+              if (s_done[x] || (x == 1 && !has_b)) continue;
+              const int b = n_sx[x] & 1;
+              if (n_sx[x] >= 2 && !mbar_test(&B->s_free[x][b], ((n_sx[x] >> 1) - 1) & 1)) continue;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff_q = (kk >> 2) * Cfg::HALF_Q + (kk & 3) * 32;
+                const uint32_t koff_k = (kk >> 2) * Cfg::HALF_KV + (kk & 3) * 32;
+                mma_bf16_ss(tmem + Cfg::tm_s(x, b),
+                            smem_desc_sw128(q_base + x * Cfg::QT_BYTES + koff_q, 16, 1024),
+                            smem_desc_sw128(k_base + ks * Cfg::KV_BYTES + koff_k, 16, 1024),
+                            Cfg::IDESC_S, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(&B->s_full[x][b]);
+              ++n_sx[x];
+              s_done[x] = true;
+              progress = true;
             }
-            mma_commit(&B->s_full[st]);
-            mma_commit(&B->k_empty[st]);
-            if (++ts == ntk_s) {            // last S of this item: Q may be replaced
-              mma_commit(&B->q_empty);
-              ws += grid;
-              ++n_s;
-              ts = 0;
-              ntk_s = ntk_next;
-              ntk_next = ws + grid < total ? (P.items[ws + grid].packed >> 8) : 0;
-              q_ok = false;
+            if (s_done[0] && (s_done[1] || !has_b)) {
+              mma_commit(&B->k_empty[ks]);
+              if (++ts == (pk_s >> 9)) {         // last S of this item: Q may be replaced
+                mma_commit(&B->q_empty);
+                ws += grid;
+                ++n_s;
+                ts = 0;
+                pk_s = pk_next;
+                pk_next = ws + grid < total ? P.items[ws + grid].packed : 0;
+                q_ok = false;
+              }
+              ++gs;
+              s_done[0] = s_done[1] = false;
             }
-            ++gs;
-            progress = true;
           }
         }
         if (gp < gs) {
           const int vs = static_cast<int>(gp % 3);
-          if (mbar_test(&B->p_full, gp & 1) && mbar_test(&B->v_full[vs], (gp / 3) & 1)) {
-            tc_fence_after();
+          const bool has_b = (pk_p & 0x1FF) > Cfg::BM;
+          if (mbar_test(&B->v_full[vs], (gp / 3) & 1)) {
 #pragma unroll
-            for (int kk = 0; kk < Cfg::BN / 16; ++kk) {
-              // A = P [128 q x 16 keys] in TMEM; B = V [16 keys x D] in smem, MN-major
-              const uint64_t b = smem_desc_sw128(v_base + vs * Cfg::KV_BYTES + kk * 2048,
-                                                 Cfg::HALF_KV, 1024);
-              mma_bf16_ts(tmem + Cfg::TM_O, tmem + Cfg::TM_P + kk * 8, b, Cfg::IDESC_PV,
-                          (tp == 0 && kk == 0) ? 0u : 1u);
+            for (int x = 0; x < 2; ++x) {
+              if (p_done[x] || (x == 1 && !has_b)) continue;
+              if (!mbar_test(&B->p_full[x], n_px[x] & 1)) continue;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < Cfg::BN / 16; ++kk) {
+                // A = P_x [128 q x 16 keys], K-major; B = V [16 keys x D], MN-major
+                mma_bf16_ss(tmem + Cfg::tm_o(x),
+                            smem_desc_sw128(p_base + x * Cfg::P_BYTES + kk * 32, 16, 1024),
+                            smem_desc_sw128(v_base + vs * Cfg::KV_BYTES + kk * 2048, Cfg::HALF_KV, 1024),
+                            Cfg::IDESC_PV, (tp == 0 && kk == 0) ? 0u : 1u);
+              }
+              mma_commit(&B->o_full[x]);
+              ++n_px[x];
+              p_done[x] = true;
+              progress = true;
             }
-            mma_commit(&B->o_full);
-            mma_commit(&B->v_empty[vs]);
-            if (++tp == ntk_p) {
-              wp += grid;
-              tp = 0;
-              ntk_p = wp < total ? (P.items[wp].packed >> 8) : 0;
+            if (p_done[0] && (p_done[1] || !has_b)) {
+              mma_commit(&B->v_empty[vs]);
+              if (++tp == (pk_p >> 9)) {
+                wp += grid;
+                tp = 0;
+                pk_p = wp < total ? P.items[wp].packed : 0;
+              }
+              ++gp;
+              p_done[0] = p_done[1] = false;
             }
-            ++gp;
-            progress = true;
           }
         }
         if (progress) {
@@ -412,45 +461,53 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // Thread `row` owns TMEM lane `row`: one query row of S and of O.
-    // Probabilities are taken against a reference max m_ref that is raised
-    // only when a tile's max exceeds it by more than kRescaleLog2; O (in
-    // TMEM) and l are rescaled then.  P values stay below 2^kRescaleLog2.
+    // Group x = warp / 4 owns query tile x of every item; thread `row` owns
+    // TMEM lane `row` (one query row of S_x and O_x).  Probabilities are taken
+    // against a reference max m_ref that is raised only when a tile's max
+    // exceeds it by more than kRescaleLog2; O_x (in TMEM) and l are rescaled
+    // then.  P values stay below 2^kRescaleLog2.
     constexpr float kRescaleLog2 = 8.f;
-    const int row = threadIdx.x;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t o_addr = tmem + lane_off + Cfg::TM_O;
+    const int x = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t o_addr = tmem + lane_off + Cfg::tm_o(x);
+    uint8_t *sPx = sP + x * Cfg::P_BYTES;
     const float sl2 = P.scale_log2;
-    uint32_t g = 0, s_iter = 0, pv_iter = 0;
+    uint32_t g = 0, n_s = 0, n_o = 0;
     AttnItem next_it = blockIdx.x < total ? P.items[blockIdx.x] : AttnItem{0, 0, 0, 0};
-    for (int w = blockIdx.x; w < total && !warp_aborted(B); w += gridDim.x) {
+    for (int w = blockIdx.x; w < total && !warp_aborted(B); w += grid) {
       const AttnItem it = next_it;
-      if (w + static_cast<int>(gridDim.x) < total) next_it = P.items[w + gridDim.x];  // prefetch
-      const int ntk = it.packed >> 8;
-      const int nrows = it.packed & 0xFF;
+      if (w + grid < total) next_it = P.items[w + grid];  // prefetch
+      const int ntk = it.packed >> 9;
+      const int rows_total = it.packed & 0x1FF;
+      const int nrows = x == 0 ? min(rows_total, Cfg::BM) : rows_total - Cfg::BM;
+      if (nrows <= 0) {          // this item has no tile B
+        g += ntk;
+        continue;
+      }
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int t = 0; t < ntk; ++t, ++g, ++s_iter) {
+      for (int t = 0; t < ntk; ++t, ++g) {
         const int st = static_cast<int>(g % 3);
         const uint32_t ph = (g / 3) & 1;
-        const uint32_t sb = s_iter & 1;
-        if (!attn_warp_wait(B, &B->s_full[sb], (s_iter >> 1) & 1, ns, SITE_ATTN_SOFTMAX) ||
+        const int sb = n_s & 1;
+        if (!attn_warp_wait(B, &B->s_full[x][sb], (n_s >> 1) & 1, ns, SITE_ATTN_SOFTMAX) ||
             !attn_warp_wait(B, &B->meta_full[st], ph, ns, SITE_ATTN_SOFTMAX)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t mk[4] = {B->meta[st][0], B->meta[st][1], B->meta[st][2], B->meta[st][3]};
-        const uint32_t s_addr = tmem + lane_off + Cfg::TM_S + sb * 128;
-        float sv[4][32];
-        tmem_ld128_sync(s_addr, reinterpret_cast<float(&)[128]>(sv));
+        const uint32_t mk[2] = {B->meta[st][0], B->meta[st][1]};
+        float sv[2][32];
+        tmem_ld64_sync(tmem + lane_off + Cfg::tm_s(x, sb), reinterpret_cast<float(&)[64]>(sv));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B->s_free[sb]);   // S buffer may be overwritten now
+        if (lane == 0) mbar_arrive(&B->s_free[x][sb]);   // S buffer may be overwritten now
+        ++n_s;
         // masked scaled scores (log2 domain) and tile max; the mask is warp-uniform
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           if (mk[c] == 0xFFFFFFFFu) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -471,24 +528,24 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           alpha = ex2_approx(m_ref - mt);
           m_ref = mt;
         }
-        // probabilities -> bf16 pairs (key 2j in the low half of column j), row sum
+        // probabilities -> bf16 pairs, row sum
         float rs2[2] = {0.f, 0.f};
-        uint32_t packed[4][16];
+        uint32_t packed[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float p0 = ex2_approx(sv[c][e] - m_ref);
             const float p1 = ex2_approx(sv[c][e + 1] - m_ref);
             rs2[0] += p0;
             rs2[1] += p1;
-            packed[c][e >> 1] = pack_bf16x2(p0, p1);
+            packed[c * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
           }
         }
-        if (t >= 1) {  // PV(t-1) must be done before P and O are touched
-          if (!attn_warp_wait(B, &B->o_full, pv_iter & 1, ns, SITE_ATTN_SOFTMAX)) { ok = false; break; }
+        if (t >= 1) {  // PV_x(t-1) must be done before P_x and O_x are touched
+          if (!attn_warp_wait(B, &B->o_full[x], n_o & 1, ns, SITE_ATTN_SOFTMAX)) { ok = false; break; }
           tc_fence_after();
-          ++pv_iter;
+          ++n_o;
           if (__any_sync(0xffffffffu, alpha != 1.f)) {   // rescale O rows in TMEM
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -502,48 +559,54 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
         l = l * alpha + (rs2[0] + rs2[1]);
-        tmem_st64(tmem + lane_off + Cfg::TM_P, reinterpret_cast<const uint32_t(&)[64]>(packed));
-        tmem_st_wait();
+        // P row: 64 keys = one 128-byte swizzle row (K-major, 16-byte chunks ^ row % 8)
+        uint8_t *prow = sPx + row * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t chunk = u ^ (row & 7);
+          *reinterpret_cast<uint4 *>(prow + chunk * 16) =
+              make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B->p_full);
+        if (lane == 0) mbar_arrive(&B->p_full[x]);
       }
       if (!ok) break;
-      if (ntk > 0) {
-        if (!attn_warp_wait(B, &B->o_full, pv_iter & 1, ns, SITE_ATTN_SOFTMAX)) break;
-        tc_fence_after();
-        ++pv_iter;
-        const float inv = 1.f / l;
-        const size_t grow = static_cast<size_t>(it.h) * P.N + it.q0 + row;
-        uint4 *dst = reinterpret_cast<uint4 *>(P.op + grow * D);
+      if (!attn_warp_wait(B, &B->o_full[x], n_o & 1, ns, SITE_ATTN_SOFTMAX)) break;
+      tc_fence_after();
+      ++n_o;
+      const float inv = 1.f / l;
+      const size_t grow = static_cast<size_t>(it.h) * P.N + it.q0 + x * Cfg::BM + row;
+      uint4 *dst = reinterpret_cast<uint4 *>(P.op + grow * D);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float ov[32];
-          tmem_ld32_sync(o_addr + c * 32, ov);
-          if (row < nrows) {
+      for (int c = 0; c < D / 32; ++c) {
+        float ov[32];
+        tmem_ld32_sync(o_addr + c * 32, ov);
+        if (row < nrows) {
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8)
-              dst[c * 4 + v8] = make_uint4(pack_bf16x2(ov[8 * v8] * inv, ov[8 * v8 + 1] * inv),
-                                           pack_bf16x2(ov[8 * v8 + 2] * inv, ov[8 * v8 + 3] * inv),
-                                           pack_bf16x2(ov[8 * v8 + 4] * inv, ov[8 * v8 + 5] * inv),
-                                           pack_bf16x2(ov[8 * v8 + 6] * inv, ov[8 * v8 + 7] * inv));
-          }
+          for (int v8 = 0; v8 < 4; ++v8)
+            dst[c * 4 + v8] = make_uint4(pack_bf16x2(ov[8 * v8] * inv, ov[8 * v8 + 1] * inv),
+                                         pack_bf16x2(ov[8 * v8 + 2] * inv, ov[8 * v8 + 3] * inv),
+                                         pack_bf16x2(ov[8 * v8 + 4] * inv, ov[8 * v8 + 5] * inv),
+                                         pack_bf16x2(ov[8 * v8 + 6] * inv, ov[8 * v8 + 7] * inv));
         }
-        tc_fence_before();
-        if (row < nrows && P.lse) P.lse[grow] = (m_ref + log2f(l)) * 0.69314718055994531f;
       }
+      tc_fence_before();
+      if (row < nrows && P.lse) P.lse[grow] = (m_ref + log2f(l)) * 0.69314718055994531f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == Cfg::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TM_COLS);
   }
 }
 
 // ------------------------------------------------------------------ planning
-// Per (head, q-cluster): number of 128-row q-tiles and of 128-key tiles.
+// Per (head, q-cluster): number of work items (256 query rows each) and of
+// 64-key tiles per item.
 __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
                                        const int32_t *__restrict__ k_off,
                                        const int32_t *__restrict__ sel_count,
@@ -556,25 +619,37 @@ __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
   const int cnt = sel_count[idx];
   const int32_t *cols = sel_cols + static_cast<size_t>(idx) * Ck;
   const int32_t *ko = k_off + static_cast<size_t>(h) * (Ck + 1);
-  int slots = 0;
+  // Selected k-clusters whose row ranges touch (consecutive ids, or ids with
+  // only empty clusters between them) form one run: slots are counted per
+  // run, exactly as the attention kernel's item loader merges them.
+  int slots = 0, run_end = -1, run_len = 0;
   for (int c = 0; c < cnt; ++c) {
     const int j = cols[c];
     if (j < 0 || j >= Ck) {
       record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
       continue;
     }
-    slots += (ko[j + 1] - ko[j] + 7) >> 3;
+    const int r0 = ko[j], len = ko[j + 1] - r0;
+    if (len <= 0) continue;
+    if (r0 == run_end) {
+      run_len += len;
+    } else {
+      slots += (run_len + 7) >> 3;
+      run_len = len;
+    }
+    run_end = r0 + len;
   }
-  int qt = nq > 0 ? (nq + 127) >> 7 : 0;
+  slots += (run_len + 7) >> 3;
+  int qt = nq > 0 ? (nq + kItemRows - 1) / kItemRows : 0;
   if (qt > 0 && slots == 0) {
     record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
     qt = 0;
   }
   qtiles[idx] = qt;
-  ktiles[idx] = (slots + 15) >> 4;
+  ktiles[idx] = (slots + kSlotsPerTile - 1) / kSlotsPerTile;
 }
 
-// Single block: one AttnItem per q-tile, ordered for the persistent kernel.
+// Single block: one AttnItem per 256 query rows, ordered for the persistent kernel.
 // Items are sorted by key-tile count, longest first (a counting sort over
 // kAttnBuckets buckets), and the sorted list is laid out in "snake" order:
 // rank r goes to round k = r / grid, slot j = r % grid, reversed on odd
@@ -641,8 +716,8 @@ __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
       const int round = rank / grid, slot = rank % grid;
       const int in_round = min(grid, n_items - round * grid);   // the last round may be partial
       const int pos = round * grid + ((round & 1) ? in_round - 1 - slot : slot);
-      const int q0 = row0 + t * 128;
-      items[pos] = AttnItem{h, i, q0, min(128, row1 - q0) | (kt << 8)};
+      const int q0 = row0 + t * kItemRows;
+      items[pos] = AttnItem{h, i, q0, min(kItemRows, row1 - q0) | (kt << 9)};
     }
   }
 }

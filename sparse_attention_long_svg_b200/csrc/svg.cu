@@ -131,7 +131,7 @@ AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
   w.num_items = c.take<int32_t>(1);
   w.qtiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.ktiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
-  w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + 127) / 128 + Cq));
+  w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + kItemRows - 1) / kItemRows + Cq));
   *bytes = c.used;
   return w;
 }
