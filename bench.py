@@ -15,6 +15,7 @@ layers processed by all ranks, divided by the max-over-ranks device time of
 the timed steps; ms_per_step is ms per layer.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl svg|reference]
+                  [--heads H] [--no-cpu-baseline]
 
 Multi-GPU (one process per GPU, torchrun): every rank runs its own layer
 (heads are independent problems), no collective on the data path; the only
@@ -191,19 +192,20 @@ def run_reference(args, wl):
     return 0
 
 
-def workload_config(wl, n_gpus):
-    return {"workload": wl.name, "heads": wl.heads, "tokens": wl.tokens, "grid": list(wl.grid),
+def workload_config(wl, n_gpus, heads=None):
+    heads = heads or wl.heads
+    return {"workload": wl.name, "heads": heads, "tokens": wl.tokens, "grid": list(wl.grid),
             "head_dim": wl.head_dim, "cq": wl.cq, "ck": wl.ck, "kmeans_iters": wl.iters, "top_p": wl.top_p[0],
             "layers_per_step_per_gpu": 1, "parallelism": f"dp{n_gpus} (independent layers per GPU)",
             "l2": "inputs larger than L2 (Q/K/V bf16 = %.0f MB > 126 MB); no flush" %
-                  (3 * wl.heads * wl.tokens * wl.head_dim * 2 / 1e6)}
+                  (3 * heads * wl.tokens * wl.head_dim * 2 / 1e6)}
 
 
 # ----------------------------------------------------------------------------- GPU leg
 
 def kernel_launches_per_step(wl) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
-    per_kmeans = 2 + 7 * wl.iters            # split, |x|^2 + T x (assign, refine, hist, scan, scatter, accum, finalize)
+    per_kmeans = 2 + 4 * wl.iters            # split, |x|^2 + T x (assign, refine, bucket, accumulate)
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
     return 2 * per_kmeans + 2 * per_permute + 1 + 3 + 1   # select; plan x2 + attention; unpermute
 
@@ -239,7 +241,7 @@ def run_svg(args, wl):
     svg.load_library()
     peaks, peak_kind = load_peaks()
 
-    L = synth.make_layer(wl)
+    L = synth.make_layer(wl, heads=args.heads)
     BH, N, D = L.q.shape
 
     def to_dev(x):
@@ -411,7 +413,7 @@ def run_svg(args, wl):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl, world),
+            "config": workload_config(wl, world, BH),
             "attn_ms": stage_ms["attn"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
             "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
@@ -450,6 +452,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="480p-5s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svg", choices=["svg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="first H heads of the workload only (smaller case for profiler captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -60,6 +60,12 @@ typedef enum svg_status {
 /* Human-readable name of a status code (static string). */
 const char *svg_status_string(svg_status s);
 
+/* The last CUDA failure that made a call return SVG_ERR_CUDA: what failed
+ * (kernel or CUDA call) and CUDA's own message; "" if none yet.  The string
+ * belongs to the library and stays valid in the calling thread until its
+ * next call of this function. */
+const char *svg_last_cuda_error(void);
+
 /* ------------------------------------------------------------------------ k-means
  * Lloyd's k-means on every head independently (section 2(a) "Clustering":
  * Q and K are clustered independently into C_q and C_k clusters).
@@ -74,9 +80,11 @@ const char *svg_status_string(svg_status s);
  *   counts     [BH, C]    int32  out: tokens per cluster for `assign`
  *
  * One round = assign (a_n = argmin_c ||x_n - mu_c||^2, ties to the lowest c)
- * then update (mu_c = mean of its tokens, summed in fp64 in ascending token
- * order; an empty cluster keeps its centroid).  The returned centroids are
- * the means of the returned assignment.  Requires iters >= 1, 1 <= C <= N,
+ * then update (mu_c = mean of its tokens, rounded once to fp32; an empty
+ * cluster keeps its centroid).  Sums run in fp64, where every partial sum of
+ * bf16 values of ordinary range is exact, so the summation order does not
+ * change the result.  The returned centroids are the means of the returned
+ * assignment.  Requires iters >= 1, 1 <= C <= N,
  * C <= 1024.  Distances run on the tensor cores with the centroids split
  * into a bf16 high and low part (about 16 significant bits).
  */

@@ -34,6 +34,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "svg_status_string": (ctypes.c_char_p, [_I]),
     "svg_version": (ctypes.c_char_p, []),
+    "svg_last_cuda_error": (ctypes.c_char_p, []),
     "svg_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
     "svg_debug_set_fault": (None, [_I]),
     "svg_get_error": (_I, [_P]),
@@ -59,8 +60,9 @@ _lib = None
 
 
 class SvgError(RuntimeError):
-    def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        msg = f"{fn} failed: {STATUS.get(status, status)}"
+        super().__init__(f"{msg} ({detail})" if detail else msg)
         self.status = status
 
 
@@ -83,7 +85,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def _check(name: str, status: int):
     if status != 0:
-        raise SvgError(name, status)
+        detail = ""
+        if status == 4 and _lib is not None:      # SVG_ERR_CUDA: say which call failed
+            detail = (_lib.svg_last_cuda_error() or b"").decode(errors="replace")
+        raise SvgError(name, status, detail)
 
 
 def _stream(stream=None) -> ctypes.c_void_p:

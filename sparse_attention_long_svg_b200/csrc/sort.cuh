@@ -44,16 +44,9 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int32_t *__restric
 // One block of 1024 threads per head; thread c owns cluster c.
 // chunk_cnt is rewritten in place with each chunk's first output row for
 // cluster c (cluster offset + rows of that cluster in earlier chunks).
-// When `row_chunks` is given, also writes row_chunks[h][c] = exclusive prefix
-// over clusters of ceil(n_c / rows_per_chunk) (entry C = the head's total):
-// the k-means update splits every cluster into chunks of at most
-// rows_per_chunk permuted rows.
 __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t *__restrict__ chunk_cnt, int N,
                                                          int C, int nch,
-                                                         int32_t *__restrict__ offsets,
-                                                         int32_t *__restrict__ counts,
-                                                         int32_t *__restrict__ row_chunks,
-                                                         int rows_per_chunk) {
+                                                         int32_t *__restrict__ offsets) {
   __shared__ int warp_tot[32];
   const int h = blockIdx.x, c = threadIdx.x;
   int32_t *cc = chunk_cnt + static_cast<size_t>(h) * nch * C;
@@ -89,36 +82,9 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t *__restrict__ c
   const int excl = warp_tot[w] + incl - total;
   if (c < C) {
     offsets[static_cast<size_t>(h) * (C + 1) + c] = excl;
-    if (counts) counts[static_cast<size_t>(h) * C + c] = total;
     for (int k = 0; k < nch; ++k) cc[static_cast<size_t>(k) * C + c] += excl;
   }
   if (c == 0) offsets[static_cast<size_t>(h) * (C + 1) + C] = N;
-  if (row_chunks == nullptr) return;
-  // second scan: chunks of at most rows_per_chunk rows per cluster
-  __syncthreads();
-  const int nck = c < C ? (total + rows_per_chunk - 1) / rows_per_chunk : 0;
-  int inc2 = nck;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, inc2, o);
-    if (lane >= o) inc2 += y;
-  }
-  if (lane == 31) warp_tot[w] = inc2;
-  __syncthreads();
-  if (w == 0) {
-    int t = warp_tot[lane];
-    int ti = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, ti, o);
-      if (lane >= o) ti += y;
-    }
-    warp_tot[lane] = ti - t;
-  }
-  __syncthreads();
-  const int ex2 = warp_tot[w] + inc2 - nck;
-  if (c < C) row_chunks[static_cast<size_t>(h) * (C + 1) + c] = ex2;
-  if (c == C - 1) row_chunks[static_cast<size_t>(h) * (C + 1) + C] = ex2 + nck;
 }
 
 // One warp per chunk: stable ranks inside each 32-token group via match_any.

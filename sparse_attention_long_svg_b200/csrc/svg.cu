@@ -26,12 +26,20 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-inline svg_status cuda_status(cudaError_t e) {
+// Text of the last CUDA failure a call reported (what failed and CUDA's message).
+char g_cuda_error[256] = "";
+std::mutex g_cuda_error_mu;
+
+inline svg_status cuda_status(cudaError_t e, const char *what = "CUDA call") {
   if (e == cudaSuccess) return SVG_OK;
+  std::lock_guard<std::mutex> lock(g_cuda_error_mu);
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s", what, cudaGetErrorString(e));
   return SVG_ERR_CUDA;
 }
 
-inline svg_status launch_status() { return cuda_status(cudaGetLastError()); }
+inline svg_status launch_status(const char *what = "kernel launch") {
+  return cuda_status(cudaGetLastError(), what);
+}
 
 // --------------------------------------------------------------- tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -77,8 +85,9 @@ int num_sms() {
 
 template <typename F>
 bool set_smem(F kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(bytes)) == cudaSuccess;
+  return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(bytes)),
+                     "shared-memory size attribute") == SVG_OK;
 }
 
 // --------------------------------------------------------------- workspace carving
@@ -100,23 +109,29 @@ struct KmeansWs {
   float *norms, *xnorm;
   __nv_bfloat16 *hi, *lo;
   KmTie *ties;
-  int32_t *perm, *offsets, *chunk, *row_chunks, *num_ties;
+  KmChunk *chunks;
+  int32_t *bucket, *offsets, *counters, *num_chunks, *num_ties;
+  int32_t *sizes(int BH, int C) const { return counters; }
+  int32_t *cursor(int BH, int C) const { return counters + static_cast<size_t>(BH) * C; }
+  int32_t *arrive(int BH, int C) const { return counters + 2 * static_cast<size_t>(BH) * C; }
 };
 KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
   Carve c{static_cast<uint8_t *>(ws)};
   KmeansWs w;
   const size_t cp = static_cast<size_t>(BH) * kmeans_cpad(C);
-  w.partial = c.take<double>(static_cast<size_t>(BH) * max_accum_chunks(N, C) * D);
-  w.row_chunks = c.take<int32_t>(static_cast<size_t>(BH) * (C + 1));
+  const size_t maxch = static_cast<size_t>(BH) * max_accum_chunks(N, C);
+  w.partial = c.take<double>(maxch * D);
+  w.chunks = c.take<KmChunk>(maxch);
+  w.num_chunks = c.take<int32_t>(BH);
   w.xnorm = c.take<float>(static_cast<size_t>(BH) * N);
   w.ties = c.take<KmTie>(static_cast<size_t>(BH) * N);
   w.num_ties = c.take<int32_t>(1);
   w.norms = c.take<float>(cp);
   w.hi = c.take<__nv_bfloat16>(cp * D);
   w.lo = c.take<__nv_bfloat16>(cp * D);
-  w.perm = c.take<int32_t>(static_cast<size_t>(BH) * N);
+  w.bucket = c.take<int32_t>(static_cast<size_t>(BH) * N);
   w.offsets = c.take<int32_t>(static_cast<size_t>(BH) * (C + 1));
-  w.chunk = c.take<int32_t>(static_cast<size_t>(BH) * num_chunks(N) * C);
+  w.counters = c.take<int32_t>(3 * static_cast<size_t>(BH) * C);   // sizes, cursors, arrivals
   *bytes = c.used;
   return w;
 }
@@ -142,10 +157,10 @@ bool sizes_ok(int BH, int N) {
 
 // Stable counting sort of assign[BH,N] by cluster: perm, offsets (and counts).
 svg_status run_sort(const int32_t *assign, int BH, int N, int C, int32_t *perm, int32_t *offsets,
-                    int32_t *counts, int32_t *chunk, cudaStream_t s, int32_t *row_chunks = nullptr) {
+                    int32_t *chunk, cudaStream_t s) {
   const int nch = num_chunks(N);
   sort_hist_kernel<<<dim3(nch, BH), 256, 0, s>>>(assign, N, C, chunk);
-  sort_scan_kernel<<<BH, 1024, 0, s>>>(chunk, N, C, nch, offsets, counts, row_chunks, kAccumRows);
+  sort_scan_kernel<<<BH, 1024, 0, s>>>(chunk, N, C, nch, offsets);
   sort_scatter_kernel<<<dim3(nch, BH), 32, 0, s>>>(assign, N, C, chunk, perm);
   return launch_status();
 }
@@ -246,6 +261,13 @@ const char *svg_status_string(svg_status s) {
   return "SVG_ERR_UNKNOWN";
 }
 
+const char *svg_last_cuda_error(void) {
+  std::lock_guard<std::mutex> lock(g_cuda_error_mu);
+  static thread_local char copy[sizeof(g_cuda_error)];
+  std::memcpy(copy, g_cuda_error, sizeof(copy));
+  return copy;
+}
+
 const char *svg_version(void) { return "svg-b200 0.1 (sm_100a)"; }
 
 void svg_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
@@ -290,17 +312,20 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
       !make_map_bf16(&mlo, w.lo, static_cast<uint64_t>(BH) * Cpad, D, 128))
     return SVG_ERR_CUDA;
   kmeans_split_kernel<<<dim3((Cpad + 7) / 8, BH), 256, 0, s>>>(centroids, C, Cpad, D, w.hi, w.lo,
-                                                              w.norms, w.num_ties);
+                                                              w.norms, w.num_ties, w.counters);
+  if (launch_status("kmeans_split_kernel") != SVG_OK) return SVG_ERR_CUDA;
   const size_t tokens = static_cast<size_t>(BH) * N;
-  const unsigned xnb = static_cast<unsigned>((tokens + 255) / 256);
+  const unsigned xnb = static_cast<unsigned>((tokens * (D / 8) + 255) / 256);
   if (D == 128)
     kmeans_xnorm_kernel<128><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
   else
     kmeans_xnorm_kernel<64><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
+  if (launch_status("kmeans_xnorm_kernel") != SVG_OK) return SVG_ERR_CUDA;
   const int units = BH * ((N + 127) / 128);
   const int ga = units < num_sms() ? units : num_sms();
-  const dim3 gu((C + 7) / 8, BH);
-  const dim3 gacc((max_accum_chunks(N, C) + 7) / 8, BH);
+  const dim3 gb((N + 1023) / 1024, BH);
+  const dim3 gacc(max_accum_chunks(N, C), BH);
+  int32_t *sizes = w.sizes(BH, C), *cursor = w.cursor(BH, C), *arrive = w.arrive(BH, C);
   if (D == 128) {
     if (!set_smem(kmeans_assign_tc_kernel<128>, KmCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
   } else {
@@ -311,30 +336,33 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
     if (pe) cudaEventRecord(pe[0], s);
     if (D == 128)
       kmeans_assign_tc_kernel<128><<<ga, KmCfg<128>::THREADS, KmCfg<128>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
+          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, sizes, w.ties, w.num_ties,
+          g_wait_ns);
     else
       kmeans_assign_tc_kernel<64><<<ga, KmCfg<64>::THREADS, KmCfg<64>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, w.ties, w.num_ties, g_wait_ns);
+          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, sizes, w.ties, w.num_ties,
+          g_wait_ns);
+    if (launch_status("kmeans_assign_tc_kernel") != SVG_OK) return SVG_ERR_CUDA;
     if (pe) cudaEventRecord(pe[1], s);
     if (D == 128)
       kmeans_refine_kernel<128><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
-                                                              w.num_ties, assign);
+                                                              w.num_ties, assign, sizes);
     else
       kmeans_refine_kernel<64><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
-                                                             w.num_ties, assign);
-    svg_status st = run_sort(assign, BH, N, C, w.perm, w.offsets, counts, w.chunk, s, w.row_chunks);
-    if (st != SVG_OK) return st;
-    if (D == 128) {
-      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, w.offsets, w.row_chunks,
-                                                    w.partial);
-      kmeans_finalize_kernel<128><<<gu, 256, 0, s>>>(N, C, Cpad, w.offsets, w.row_chunks, w.partial,
-                                                     centroids, w.hi, w.lo, w.norms, w.num_ties);
-    } else {
-      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, w.perm, w.offsets, w.row_chunks,
-                                                   w.partial);
-      kmeans_finalize_kernel<64><<<gu, 256, 0, s>>>(N, C, Cpad, w.offsets, w.row_chunks, w.partial,
+                                                             w.num_ties, assign, sizes);
+    if (launch_status("kmeans_refine_kernel") != SVG_OK) return SVG_ERR_CUDA;
+    kmeans_bucket_kernel<<<gb, 1024, 0, s>>>(assign, N, C, sizes, cursor, w.bucket, w.offsets,
+                                             counts, w.chunks, w.num_chunks);
+    if (launch_status("kmeans_bucket_kernel") != SVG_OK) return SVG_ERR_CUDA;
+    if (D == 128)
+      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
+                                                    w.num_chunks, w.partial, arrive, sizes, cursor,
                                                     centroids, w.hi, w.lo, w.norms, w.num_ties);
-    }
+    else
+      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
+                                                   w.num_chunks, w.partial, arrive, sizes, cursor,
+                                                   centroids, w.hi, w.lo, w.norms, w.num_ties);
+    if (launch_status("kmeans_accum_kernel") != SVG_OK) return SVG_ERR_CUDA;
   }
   return launch_status();
 }
@@ -363,7 +391,7 @@ svg_status svg_permute(const int32_t *assign, int BH, int N, int C, int32_t *per
   if (!aligned(ws, 256)) return SVG_ERR_INVALID_ARG;
   if (ws_bytes < svg_permute_workspace_size(BH, N, C)) return SVG_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  svg_status st = run_sort(assign, BH, N, C, perm, offsets, nullptr, static_cast<int32_t *>(ws), s);
+  svg_status st = run_sort(assign, BH, N, C, perm, offsets, static_cast<int32_t *>(ws), s);
   if (st != SVG_OK || ntensors == 0) return st;
   return run_row_move(true, ntensors, src, dst, perm, BH, N, D, s);
 }

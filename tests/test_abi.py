@@ -43,6 +43,7 @@ def test_status_strings(lib):
     for code, name in svg.STATUS.items():
         assert lib.svg_status_string(code).decode() == name
     assert lib.svg_version().decode().startswith("svg-b200")
+    assert lib.svg_last_cuda_error().decode() == ""      # no CUDA call has failed in this process
 
 
 def test_workspace_sizes_are_positive_and_monotone(lib):
