@@ -16,7 +16,7 @@
 //   atomic cursors, so the order inside a cluster is arbitrary).  The first
 //   block of each head also publishes the offsets, the sizes and a table of
 //   accumulation chunks (at most kAccumRows rows of one cluster each).
-// kmeans_accum_kernel: one block per chunk sums its rows in fp64; a cluster
+// kmeans_accum_kernel: one warp per chunk sums its rows in fp64; a cluster
 //   with one chunk is finalised at once, otherwise the last of its chunks to
 //   arrive adds the chunks' partial sums and finalises.  Finalising writes the
 //   new fp32 centroid, its bf16 hi/lo split and squared norm for the next
@@ -27,7 +27,8 @@
 
 namespace svg {
 
-constexpr int kAccumRows = 256;
+constexpr int kAccumRows = 128;
+constexpr int kBucketTokens = 4;   // tokens per thread of the bucket kernel
 
 __host__ __device__ inline int max_accum_chunks(int N, int C) {
   return (N + kAccumRows - 1) / kAccumRows + C;
@@ -68,7 +69,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *t
   return r;
 }
 
-// grid (ceil(N / 1024), BH), 1024 threads.
+// grid (ceil(N / (1024 * kBucketTokens)), BH), 1024 threads; thread t of a
+// block takes tokens base + t + 1024 k, k < kBucketTokens.
 // counts [BH, C]: sizes of this round's clusters (from the assign step);
 // cursor [BH, C]: zero on entry, the sizes on exit.
 __global__ void __launch_bounds__(1024) kmeans_bucket_kernel(
@@ -80,6 +82,14 @@ __global__ void __launch_bounds__(1024) kmeans_bucket_kernel(
   __shared__ int warp_tot[32];
   __shared__ int s_total;
   const int h = blockIdx.y, t = threadIdx.x, lane = t & 31;
+  const int32_t *ah = assign + static_cast<size_t>(h) * N;
+  const int n_base = blockIdx.x * blockDim.x * kBucketTokens + t;
+  int a[kBucketTokens];
+#pragma unroll
+  for (int k = 0; k < kBucketTokens; ++k) {   // issued before the scan so they overlap it
+    const int n = n_base + k * static_cast<int>(blockDim.x);
+    a[k] = n < N ? ah[n] : -1;
+  }
   const int cnt = t < C ? counts[static_cast<size_t>(h) * C + t] : 0;
   const int excl = block_exclusive_scan(cnt, warp_tot, &s_total);
   if (t < C) s_off[t] = excl;
@@ -98,27 +108,89 @@ __global__ void __launch_bounds__(1024) kmeans_bucket_kernel(
     if (t == 0) num_chunks[h] = s_total;
   }
   __syncthreads();
-  const int n = blockIdx.x * blockDim.x + t;
-  const int a = n < N ? assign[static_cast<size_t>(h) * N + n] : -1;
-  const bool ok = a >= 0 && a < C;
-  if (n < N && !ok) record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);
-  const unsigned live = __ballot_sync(0xffffffffu, ok);
-  if (ok) {
-    const unsigned peers = __match_any_sync(live, a);
-    const int leader = __ffs(peers) - 1;
-    int base = 0;
-    if (lane == leader) base = atomicAdd(cursor + static_cast<size_t>(h) * C + a, __popc(peers));
-    base = __shfl_sync(live, base, leader);
-    const int pos = s_off[a] + base + __popc(peers & ((1u << lane) - 1u));
-    if (pos < N) {
-      bucket[static_cast<size_t>(h) * N + pos] = n;
-    } else {
-      record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);   // sizes and assignment disagree
+  int base[kBucketTokens];
+  unsigned peers[kBucketTokens];
+#pragma unroll
+  for (int k = 0; k < kBucketTokens; ++k) {    // reserve: one atomic per cluster of a warp
+    const int n = n_base + k * static_cast<int>(blockDim.x);
+    const bool ok = a[k] >= 0 && a[k] < C;
+    if (n < N && !ok) record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);
+    const unsigned live = __ballot_sync(0xffffffffu, ok);
+    peers[k] = 0;
+    base[k] = 0;
+    if (ok) {
+      peers[k] = __match_any_sync(live, a[k]);
+      if (lane == __ffs(peers[k]) - 1)
+        base[k] = atomicAdd(cursor + static_cast<size_t>(h) * C + a[k], __popc(peers[k]));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kBucketTokens; ++k) {    // place
+    const bool ok = peers[k] != 0;
+    const unsigned live = __ballot_sync(0xffffffffu, ok);
+    if (ok) {
+      const int b0 = __shfl_sync(live, base[k], __ffs(peers[k]) - 1);
+      const int pos = s_off[a[k]] + b0 + __popc(peers[k] & ((1u << lane) - 1u));
+      if (pos < N) {
+        bucket[static_cast<size_t>(h) * N + pos] = n_base + k * static_cast<int>(blockDim.x);
+      } else {
+        record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);   // sizes and assignment disagree
+      }
     }
   }
 }
 
-// grid (max_accum_chunks(N, C), BH), 256 threads (8 warps).
+// Writes cluster c's new centroid from its fp64 row sum: lanes l < D/8 hold
+// channels 8l .. 8l+7 of the sum.  Also clears the cluster's counters.
+template <int D>
+__device__ __forceinline__ void kmeans_finalize_cluster(const double (&sum)[8], int lane, int h,
+                                                        int c, int C, int Cpad, int n_c,
+                                                        float *__restrict__ mu,
+                                                        __nv_bfloat16 *__restrict__ hi,
+                                                        __nv_bfloat16 *__restrict__ lo,
+                                                        float *__restrict__ norms,
+                                                        int32_t *__restrict__ counts_ws,
+                                                        int32_t *__restrict__ cursor) {
+  constexpr int LPR = D / 8;
+  float sq = 0.f;
+  if (lane < LPR) {
+    float out[8];
+    uint32_t hp[4], lp[4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      out[e] = static_cast<float>(sum[e] / n_c);
+      sq = fmaf(out[e], out[e], sq);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(out[e]), h1 = __float2bfloat16_rn(out[e + 1]);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(out[e] - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(out[e + 1] - __bfloat162float(h1));
+      hp[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+      lp[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+    }
+    float4 *m = reinterpret_cast<float4 *>(mu + (static_cast<size_t>(h) * C + c) * D + lane * 8);
+    m[0] = make_float4(out[0], out[1], out[2], out[3]);
+    m[1] = make_float4(out[4], out[5], out[6], out[7]);
+    const size_t srow = (static_cast<size_t>(h) * Cpad + c) * D + lane * 8;
+    *reinterpret_cast<uint4 *>(hi + srow) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+    *reinterpret_cast<uint4 *>(lo + srow) = make_uint4(lp[0], lp[1], lp[2], lp[3]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if (lane == 0) {
+    norms[static_cast<size_t>(h) * Cpad + c] = sq;
+    counts_ws[static_cast<size_t>(h) * C + c] = 0;    // counters of the next round
+    cursor[static_cast<size_t>(h) * C + c] = 0;
+  }
+}
+
+// grid (ceil(max_accum_chunks(N, C) / 8), BH), 256 threads: warp w of block b
+// sums chunk j = 8 b + w.  A row is D/8 lanes x 16 bytes; a warp load covers
+// 32 / (D/8) rows, UNROLL loads are in flight.  Lane l keeps channels
+// 8 (l % (D/8)) .. +7 in fp64.
 template <int D>
 __global__ void __launch_bounds__(256) kmeans_accum_kernel(
     const __nv_bfloat16 *__restrict__ x, int N, int C, int Cpad, const int32_t *__restrict__ bucket,
@@ -127,103 +199,84 @@ __global__ void __launch_bounds__(256) kmeans_accum_kernel(
     int32_t *__restrict__ arrive, int32_t *__restrict__ counts_ws, int32_t *__restrict__ cursor,
     float *__restrict__ mu, __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo,
     float *__restrict__ norms, int32_t *__restrict__ num_ties) {
-  constexpr int PER = D / 32;
-  constexpr int WARPS = 8, UNROLL = 8;
-  __shared__ double s_red[WARPS][D];
-  __shared__ float s_sq[D / 32];
-  __shared__ int s_last;
-  const int h = blockIdx.y, j = blockIdx.x;
-  if (j == 0 && h == 0 && threadIdx.x == 0) *num_ties = 0;   // the refine step of this round is done
+  constexpr int LPR = D / 8;           // lanes per row
+  constexpr int RPL = 32 / LPR;        // rows per warp load
+  constexpr int UNROLL = 8;
+  constexpr int STEP = RPL * UNROLL;   // rows per iteration
+  const int h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  if (j == 0 && h == 0 && lane == 0) *num_ties = 0;   // the refine step of this round is done
   if (j >= num_chunks[h]) return;
   const int maxch = max_accum_chunks(N, C);
   const KmChunk ch = chunks[static_cast<size_t>(h) * maxch + j];
   const int c = ch.c;
+  const int32_t *b = bucket + static_cast<size_t>(h) * N + ch.r0;
+  const int len = ch.r1 - ch.r0;
+  const int sub = lane / LPR, q = lane % LPR;
+  const uint4 *xh = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(h) * N * D) + q;
+  double sum[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sum[e] = 0.0;
+  for (int r = 0; r < len; r += STEP) {
+    const int id = r + lane < len ? b[r + lane] : -1;   // STEP <= 32 row ids, one per lane
+    uint4 v[UNROLL];
+    bool ok[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int t = __shfl_sync(0xffffffffu, id, u * RPL + sub);
+      ok[u] = t >= 0;
+      v[u] = ok[u] ? __ldg(xh + static_cast<size_t>(t) * LPR) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      if (!ok[u]) continue;
+      const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p2[e]);
+        sum[2 * e] += static_cast<double>(f.x);
+        sum[2 * e + 1] += static_cast<double>(f.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], o);
   const int n_c = offsets[static_cast<size_t>(h) * (C + 1) + c + 1] -
                   offsets[static_cast<size_t>(h) * (C + 1) + c];
   const int nch = (n_c + kAccumRows - 1) / kAccumRows;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t *b = bucket + static_cast<size_t>(h) * N + ch.r0;
-  const __nv_bfloat16 *xh = x + static_cast<size_t>(h) * N * D + lane * PER;
-  const int len = ch.r1 - ch.r0;
-  double acc[PER];
+  if (nch > 1) {
+    double *part = partial + static_cast<size_t>(h) * maxch * D;
+    if (lane < LPR) {
+      double2 *dst = reinterpret_cast<double2 *>(part + static_cast<size_t>(j) * D + lane * 8);
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.0;
-  // warp w takes rows w, w + 8, w + 16, ...; UNROLL rows in flight per warp
-  for (int base = warp; base < len; base += WARPS * UNROLL) {
-    int id = -1;
-    if (lane < UNROLL && base + WARPS * lane < len) id = b[base + WARPS * lane];
-    int ids[UNROLL];
-    float v[UNROLL][PER];
+      for (int e = 0; e < 4; ++e) dst[e] = make_double2(sum[2 * e], sum[2 * e + 1]);
+    }
+    __threadfence();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(arrive + static_cast<size_t>(h) * C + c, 1) == nch - 1;
+    if (!__shfl_sync(0xffffffffu, last, 0)) return;
+    __threadfence();
+    if (lane < LPR) {
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      ids[u] = __shfl_sync(0xffffffffu, id, u);
-      if (ids[u] >= 0) {                       // warp-uniform
-        const __nv_bfloat16 *row = xh + static_cast<size_t>(ids[u]) * D;
-        if constexpr (PER == 4) {
-          const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(row));
-          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-          v[u][0] = f0.x; v[u][1] = f0.y; v[u][2] = f1.x; v[u][3] = f1.y;
-        } else {
-          const uint32_t raw = __ldg(reinterpret_cast<const uint32_t *>(row));
-          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw));
-          v[u][0] = f0.x; v[u][1] = f0.y;
+      for (int e = 0; e < 8; ++e) sum[e] = 0.0;
+      for (int k = 0; k < nch; ++k) {
+        const double2 *src =
+            reinterpret_cast<const double2 *>(part + static_cast<size_t>(ch.j0 + k) * D + lane * 8);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double2 d2 = __ldcg(src + e);
+          sum[2 * e] += d2.x;
+          sum[2 * e + 1] += d2.y;
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u)
-      if (ids[u] >= 0)
-#pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += static_cast<double>(v[u][e]);
+    if (lane == 0) arrive[static_cast<size_t>(h) * C + c] = 0;
   }
-#pragma unroll
-  for (int e = 0; e < PER; ++e) s_red[warp][lane * PER + e] = acc[e];
-  __syncthreads();
-  const int d = threadIdx.x;
-  double sum = 0.0;
-  if (d < D)
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) sum += s_red[w][d];
-  if (nch > 1) {
-    double *part = partial + static_cast<size_t>(h) * maxch * D;
-    if (d < D) part[static_cast<size_t>(j) * D + d] = sum;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0)
-      s_last = atomicAdd(arrive + static_cast<size_t>(h) * C + c, 1) == nch - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (d < D) {
-      sum = 0.0;
-      for (int k = 0; k < nch; ++k) sum += __ldcg(part + static_cast<size_t>(ch.j0 + k) * D + d);
-    }
-    if (threadIdx.x == 0) arrive[static_cast<size_t>(h) * C + c] = 0;
-  }
-  // finalise cluster c (n_c >= 1 here)
-  float out = 0.f;
-  if (d < D) {
-    out = static_cast<float>(sum / n_c);
-    mu[(static_cast<size_t>(h) * C + c) * D + d] = out;
-    const __nv_bfloat16 vh = __float2bfloat16_rn(out);
-    const size_t srow = (static_cast<size_t>(h) * Cpad + c) * D + d;
-    hi[srow] = vh;
-    lo[srow] = __float2bfloat16_rn(out - __bfloat162float(vh));
-  }
-  float sq = out * out;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  if (lane == 0 && warp < D / 32) s_sq[warp] = sq;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) s += s_sq[w];
-    norms[static_cast<size_t>(h) * Cpad + c] = s;
-    counts_ws[static_cast<size_t>(h) * C + c] = 0;    // counters of the next round
-    cursor[static_cast<size_t>(h) * C + c] = 0;
-  }
+  kmeans_finalize_cluster<D>(sum, lane, h, c, C, Cpad, n_c, mu, hi, lo, norms, counts_ws, cursor);
 }
 
 }  // namespace svg

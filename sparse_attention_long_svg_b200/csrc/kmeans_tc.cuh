@@ -249,11 +249,12 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
     // and runner-up with the half-chunk's first column (an equal key keeps the
     // earlier column).  When a unit has several chunks, group 1 hands its pair
     // to group 0 through shared memory and group 0 merges.
-    // Near-tie rule: a key is within 2^-14 (||x||^2 + ||mu||^2) of its score
-    // (|s| <= 2 (||x||^2 + ||mu||^2)), and the tensor-core score is within
-    // about 2^-16 (||x||^2 + ||mu||^2) of the exact one (bf16 split residual
-    // and fp32 accumulation); a runner-up within 2^-11 (||x||^2 + the larger
-    // ||mu||^2) of the best goes to the exact float32 re-check.
+    // Near-tie rule: a key is within 2^-15 |s| of its score, and the
+    // tensor-core score is within about 2^-16 (||x||^2 + ||mu||^2) of the
+    // exact one (bf16 split residual and fp32 accumulation).  A runner-up
+    // within 2^-14 (|key_1| + |key_2| + ||x||^2 + the larger ||mu||^2) of the
+    // best (twice the key term, four times the tensor-core term) goes to the
+    // exact float32 re-check.
     constexpr float kBig = 3.0e38f;
     const int grp = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
       if (live && arg2 >= 0 && arg2 < C) {
         const float xx = __ldg(xnorm + static_cast<size_t>(h) * N + n0 + row);
         const float mm = fmaxf(__ldg(nh + arg), __ldg(nh + arg2));
-        tie = second - best <= 0x1p-11f * (xx + mm);
+        tie = second - best <= 0x1p-14f * (fabsf(best) + fabsf(second) + xx + mm);
       }
       const unsigned tmask = __ballot_sync(0xffffffffu, tie);
       if (tmask) {   // warp-aggregated append to the near-tie list

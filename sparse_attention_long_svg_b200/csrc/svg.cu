@@ -323,8 +323,8 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   if (launch_status("kmeans_xnorm_kernel") != SVG_OK) return SVG_ERR_CUDA;
   const int units = BH * ((N + 127) / 128);
   const int ga = units < num_sms() ? units : num_sms();
-  const dim3 gb((N + 1023) / 1024, BH);
-  const dim3 gacc(max_accum_chunks(N, C), BH);
+  const dim3 gb((N + 1024 * kBucketTokens - 1) / (1024 * kBucketTokens), BH);
+  const dim3 gacc((max_accum_chunks(N, C) + 7) / 8, BH);
   int32_t *sizes = w.sizes(BH, C), *cursor = w.cursor(BH, C), *arrive = w.arrive(BH, C);
   if (D == 128) {
     if (!set_smem(kmeans_assign_tc_kernel<128>, KmCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
