@@ -288,24 +288,32 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
         }
         tc_fence_after();
         const float4 *nv4 = reinterpret_cast<const float4 *>(sNorm + ab * Cfg::NC);
+        const uint32_t acc_addr = tmem + lane_off + ab * Cfg::NC;
+        // 32-column pieces: the next piece's TMEM load is in flight while the
+        // current one is reduced
+        uint32_t buf[2][32];
+        tmem_ld32_start(acc_addr, buf[0]);
+        tmem_wait32(buf[0]);
+        float p1 = kBig, p2 = kBig, q1 = kBig, q2 = kBig;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float acc[64];
-          tmem_ld64_sync(tmem + lane_off + ab * Cfg::NC + half * 64, acc);
-          if (half == 1) {       // the accumulator is in registers: the MMAs may reuse it
+        for (int pc = 0; pc < 4; ++pc) {
+          if (pc < 3) {
+            tmem_ld32_start(acc_addr + (pc + 1) * 32, buf[(pc + 1) & 1]);
+          } else {               // every piece is in registers: the MMAs may reuse the buffer
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&B->acc_empty[ab]);
           }
-          float p1 = kBig, p2 = kBig, q1 = kBig, q2 = kBig;
+          const uint32_t *acc = buf[pc & 1];
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4) {
-            const float4 nv = nv4[half * 16 + c4];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 nv = nv4[pc * 8 + c4];
             const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float sc = fmaf(-2.f, acc[4 * c4 + e], nn[e]);
-              const float k = __int_as_float(__byte_perm(__float_as_int(sc), colb[c4], 0x3214 + e));
+              const float sc = fmaf(-2.f, __uint_as_float(acc[4 * c4 + e]), nn[e]);
+              const float k = __int_as_float(
+                  __byte_perm(__float_as_int(sc), colb[(pc & 1) * 8 + c4], 0x3214 + e));
               if (e & 1) {
                 q2 = fminf(q2, fmaxf(q1, k));
                 q1 = fminf(q1, k);
@@ -315,18 +323,22 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
               }
             }
           }
-          const float m1 = fminf(p1, q1);
-          const float m2 = fminf(fmaxf(p1, q1), fminf(p2, q2));
-          const int cbase = j * Cfg::NC + half * 64;
-          const int mc1 = cbase + (__float_as_int(m1) & 0xFF);
-          const int mc2 = cbase + (__float_as_int(m2) & 0xFF);
-          const bool n1 = m1 < best, n2 = m1 < second, s1 = m2 < best;
-          const float ns = n1 ? (s1 ? m2 : best) : (n2 ? m1 : second);
-          const int nsa = n1 ? (s1 ? mc2 : arg) : (n2 ? mc1 : arg2);
-          best = n1 ? m1 : best;
-          arg = n1 ? mc1 : arg;
-          second = ns;
-          arg2 = nsa;
+          if (pc & 1) {          // end of a 64-column half: merge its pair
+            const float m1 = fminf(p1, q1);
+            const float m2 = fminf(fmaxf(p1, q1), fminf(p2, q2));
+            const int cbase = j * Cfg::NC + (pc >> 1) * 64;
+            const int mc1 = cbase + (__float_as_int(m1) & 0xFF);
+            const int mc2 = cbase + (__float_as_int(m2) & 0xFF);
+            const bool n1 = m1 < best, n2 = m1 < second, s1 = m2 < best;
+            const float ns = n1 ? (s1 ? m2 : best) : (n2 ? m1 : second);
+            const int nsa = n1 ? (s1 ? mc2 : arg) : (n2 ? mc1 : arg2);
+            best = n1 ? m1 : best;
+            arg = n1 ? mc1 : arg;
+            second = ns;
+            arg2 = nsa;
+            p1 = p2 = q1 = q2 = kBig;
+          }
+          if (pc < 3) tmem_wait32(buf[(pc + 1) & 1]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&B->n_empty[ab]);
