@@ -207,7 +207,7 @@ def kernel_launches_per_step(wl) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
     per_kmeans = 2 + 4 * wl.iters            # split, |x|^2 + T x (assign, refine, bucket, accumulate)
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
-    return 2 * per_kmeans + 2 * per_permute + 1 + 3 + 1   # select; plan x2 + attention; unpermute
+    return 2 * per_kmeans + 2 * per_permute + 1 + 3       # select; plan x2 + attention (un-permute fused)
 
 
 def attention_pairs(layer, wl):
@@ -255,9 +255,9 @@ def run_svg(args, wl):
     out = torch.empty_like(q)
     p = wl.top_p[0]
     stream = torch.cuda.current_stream()
-    stage_names = ["kmeans_q", "kmeans_k", "permute", "select", "attn", "unpermute"]
+    stage_names = ["kmeans_q", "kmeans_k", "permute", "select", "attn+unpermute"]
 
-    def step(ev=None):
+    def step(ev=None):   # the un-permutation is fused into the attention kernel's store
         mu_q.copy_(mu_q0)
         mu_k.copy_(mu_k0)
         if ev:
@@ -277,12 +277,9 @@ def run_svg(args, wl):
         if ev:
             ev[4].record()
         svg.sparse_attn(layer.qp, layer.kp, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
-                        layer.sel_cols, 0.0, layer.op, workspace=layer.workspace)
+                        layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
         if ev:
             ev[5].record()
-        svg.unpermute(layer.op, layer.perm_q, out)
-        if ev:
-            ev[6].record()
 
     clocks = ClockSampler(device.index)
     clocks.__enter__()          # sampling starts with the warm-up so short runs still see load
@@ -292,7 +289,7 @@ def run_svg(args, wl):
     if svg.get_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -358,7 +355,7 @@ def run_svg(args, wl):
     # ---- rooflines of the two heavy kernels, from the live event timings
     tc_peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    attn_tflops = flops_layer / (stage_ms["attn"] * 1e-3) / 1e12
+    attn_tflops = flops_layer / (stage_ms["attn+unpermute"] * 1e-3) / 1e12
     peak_note = f"{peak_kind} bf16 sustained (kernel timed inside a multi-ms step)"
     attn_kernel_ms = attn_k_ms / max(attn_n, 1)
     attn_kernel_tflops = flops_layer / (attn_kernel_ms * 1e-3) / 1e12
@@ -391,12 +388,12 @@ def run_svg(args, wl):
                      "gbs": km_bytes / stage_ms["kmeans_k"] / 1e6},
         "permute": {"ms": stage_ms["permute"], "gbs": 6.0 * tensor_bytes / stage_ms["permute"] / 1e6},
         "select": {"ms": stage_ms["select"]},
-        "attn": {"ms": stage_ms["attn"], "tflops": attn_tflops},
-        "unpermute": {"ms": stage_ms["unpermute"], "gbs": 2.0 * tensor_bytes / stage_ms["unpermute"] / 1e6},
+        "attn+unpermute": {"ms": stage_ms["attn+unpermute"], "tflops": attn_tflops,
+                           "note": "un-permutation fused into the attention kernel's store"},
     }
-    for sname in ("kmeans_q", "kmeans_k", "permute", "unpermute"):
+    for sname in ("kmeans_q", "kmeans_k", "permute"):
         stages[sname]["hbm_frac"] = stages[sname]["gbs"] / hbm_peak
-    for sname in ("kmeans_q", "kmeans_k", "attn"):
+    for sname in ("kmeans_q", "kmeans_k", "attn+unpermute"):
         stages[sname]["tensor_frac"] = stages[sname]["tflops"] / tc_peak
 
     cpu = None
@@ -414,7 +411,7 @@ def run_svg(args, wl):
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wl, world, BH),
-            "attn_ms": stage_ms["attn"], "attn_eff_tflops": attn_tflops,
+            "attn_ms": stage_ms["attn+unpermute"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
             "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -154,6 +154,26 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
                            const int32_t *sel_count, const int32_t *sel_cols, float scale, void *op,
                            float *lse, void *ws, size_t ws_bytes, svg_stream_t stream);
 
+/* The same attention with the un-permutation (section 2(a) "Mathematical
+ * equivalence": O[perm_q[r]] = O'[r]) fused into the kernel's store: row r
+ * of a head's result goes to row perm_q[r] of o, so o is in the original token
+ * order and no permuted copy of the output exists.
+ *
+ *   perm_q  [BH, N]    int32  the Q permutation (svg_permute), required
+ *   o       [BH, N, D] bf16   out: attention output in token order; must not
+ *                             alias qp, kp or vp
+ *   lse     [BH, N]    fp32   optional out, also in token order
+ * Other arguments, the workspace and the result are those of svg_sparse_attn
+ * followed by svg_unpermute.  A perm_q entry outside [0, N) is skipped and
+ * flagged with SVG_ERR_DEVICE_CHECK.
+ */
+svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void *vp, int BH,
+                                      int N, int D, const int32_t *q_off, int Cq,
+                                      const int32_t *k_off, int Ck, const int32_t *sel_count,
+                                      const int32_t *sel_cols, float scale, const int32_t *perm_q,
+                                      void *o, float *lse, void *ws, size_t ws_bytes,
+                                      svg_stream_t stream);
+
 /* ------------------------------------------------------------------------ sparse attention, no allocation
  * No counterpart on the pages: this is a service for callers that cannot hand
  * the library a scratch buffer.  Some callers have no way to obtain device

@@ -45,6 +45,8 @@ SIGNATURES = {
     "svg_select_topp": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P, _P, _P]),
     "svg_sparse_attn_workspace_size": (_SZ, [_I, _I, _I]),
     "svg_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _SZ, _P]),
+    "svg_sparse_attn_unpermuted": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
+                                        _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "svg_sparse_attn_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P]),
     "svg_profile_enable": (_I, [_I]),
@@ -217,8 +219,12 @@ def select_topp(mu_q: torch.Tensor, n_q: torch.Tensor, mu_k: torch.Tensor, n_k: 
 
 
 def sparse_attn(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
-                want_lse: bool = False, lse=None, workspace=None, stream=None):
-    """Attention over the selected blocks of permuted Q/K/V.  Returns (op, lse or None)."""
+                want_lse: bool = False, lse=None, workspace=None, stream=None, perm_q=None):
+    """Attention over the selected blocks of permuted Q/K/V.  Returns (op, lse or None).
+
+    With ``perm_q`` (the Q permutation) the un-permutation is fused into the
+    kernel's store: ``op`` (and ``lse``) come back in the original token order.
+    """
     lib = load_library()
     for t, n in ((qp, "qp"), (kp, "kp"), (vp, "vp")):
         _need(t, n, torch.bfloat16, 3)
@@ -231,6 +237,13 @@ def sparse_attn(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.
         lse = torch.empty((BH, N), dtype=torch.float32, device=qp.device)
     if workspace is None:
         workspace = _ws(lib.svg_sparse_attn_workspace_size(BH, N, Cq), qp.device)
+    if perm_q is not None:
+        _need(perm_q, "perm_q", torch.int32, 2)
+        _check("svg_sparse_attn_unpermuted", lib.svg_sparse_attn_unpermuted(
+            _ptr(qp), _ptr(kp), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
+            _ptr(sel_cols), float(scale), _ptr(perm_q), _ptr(op), _ptr(lse), _ptr(workspace),
+            workspace.numel(), _stream(stream)))
+        return op, lse
     _check("svg_sparse_attn", lib.svg_sparse_attn(
         _ptr(qp), _ptr(kp), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
         _ptr(sel_cols), float(scale), _ptr(op), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
@@ -292,7 +305,7 @@ class LayerState:
     qp: torch.Tensor
     kp: torch.Tensor
     vp: torch.Tensor
-    op: torch.Tensor
+    op: Optional[torch.Tensor]     # permuted output; None when the un-permutation was fused
 
 
 class SvgLayer:
@@ -322,19 +335,30 @@ class SvgLayer:
                  lib.svg_sparse_attn_workspace_size(BH, N, Cq))
         self.workspace = _ws(ws, device)
 
-    def __call__(self, q, k, v, mu_q, mu_k, iters: int, p: float, scale: float = 0.0, out=None, stream=None):
+    def __call__(self, q, k, v, mu_q, mu_k, iters: int, p: float, scale: float = 0.0, out=None, stream=None,
+                 fused_unpermute: bool = True):
+        """One layer; with ``fused_unpermute`` the attention kernel stores rows in token order
+        (no permuted output copy, ``LayerState.op`` is None), else attention + svg_unpermute."""
         kmeans(q, mu_q, iters, self.assign_q, self.n_q, self.workspace, stream)
         kmeans(k, mu_k, iters, self.assign_k, self.n_k, self.workspace, stream)
         Cq, Ck = mu_q.shape[1], mu_k.shape[1]
         permute(self.assign_q, Cq, [q], [self.qp], self.perm_q, self.q_off, self.workspace, stream)
         permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace, stream)
         select_topp(mu_q, self.n_q, mu_k, self.n_k, p, scale, self.sel_count, self.sel_cols, stream)
-        sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,
-                    self.op, workspace=self.workspace, stream=stream)
-        out = unpermute(self.op, self.perm_q, out, stream)
+        if fused_unpermute:
+            if out is None:
+                out = torch.empty_like(q)
+            sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,
+                        out, workspace=self.workspace, stream=stream, perm_q=self.perm_q)
+            op = None
+        else:
+            sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,
+                        self.op, workspace=self.workspace, stream=stream)
+            out = unpermute(self.op, self.perm_q, out, stream)
+            op = self.op
         return out, LayerState(mu_q, mu_k, self.assign_q, self.assign_k, self.n_q, self.n_k, self.perm_q,
                                self.perm_k, self.q_off, self.k_off, self.sel_count, self.sel_cols, self.qp,
-                               self.kp, self.vp, self.op)
+                               self.kp, self.vp, op)
 
 
 def svg_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mu_q: torch.Tensor, mu_k: torch.Tensor,

@@ -110,6 +110,7 @@ struct AttnParams {
   const int32_t *num_items;
   __nv_bfloat16 *op;
   float *lse;
+  const int32_t *perm;   // optional: write row r of a head to row perm[r] (un-permuted output)
   int N, Cq, Ck, BH;
   float scale_log2;      // softmax scale * log2(e)
   uint64_t wait_ns;
@@ -577,13 +578,23 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       tc_fence_after();
       ++n_o;
       const float inv = 1.f / l;
-      const size_t grow = static_cast<size_t>(it.h) * P.N + it.q0 + x * Cfg::BM + row;
-      uint4 *dst = reinterpret_cast<uint4 *>(P.op + grow * D);
+      size_t grow = static_cast<size_t>(it.h) * P.N + it.q0 + x * Cfg::BM + row;
+      if (P.perm != nullptr && row < nrows) {   // un-permute fused into the store
+        const int t = P.perm[grow];
+        if (t >= 0 && t < P.N) {
+          grow = static_cast<size_t>(it.h) * P.N + t;
+        } else {
+          record_error(SVG_ERR_DEVICE_CHECK, SITE_PERMUTE_RANGE);
+          grow = static_cast<size_t>(-1);
+        }
+      }
+      const bool store = row < nrows && grow != static_cast<size_t>(-1);
+      uint4 *dst = reinterpret_cast<uint4 *>(P.op + (store ? grow : 0) * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];
         tmem_ld32_sync(o_addr + c * 32, ov);
-        if (row < nrows) {
+        if (store) {
 #pragma unroll
           for (int v8 = 0; v8 < 4; ++v8)
             dst[c * 4 + v8] = make_uint4(pack_bf16x2(ov[8 * v8] * inv, ov[8 * v8 + 1] * inv),
@@ -593,7 +604,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
       }
       tc_fence_before();
-      if (row < nrows && P.lse) P.lse[grow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (store && P.lse) P.lse[grow] = (m_ref + log2f(l)) * 0.69314718055994531f;
     }
   }
   tc_fence_before();

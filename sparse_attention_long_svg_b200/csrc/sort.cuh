@@ -52,10 +52,15 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t *__restrict__ c
   int32_t *cc = chunk_cnt + static_cast<size_t>(h) * nch * C;
   int total = 0;
   if (c < C) {
-    for (int k = 0; k < nch; ++k) {
-      int v = cc[static_cast<size_t>(k) * C + c];
-      cc[static_cast<size_t>(k) * C + c] = total;
-      total += v;
+    for (int k0 = 0; k0 < nch; k0 += 8) {   // eight loads in flight, then the running sum
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = k0 + u < nch ? cc[static_cast<size_t>(k0 + u) * C + c] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (k0 + u < nch) cc[static_cast<size_t>(k0 + u) * C + c] = total;
+        total += v[u];
+      }
     }
   }
   // exclusive scan of totals over clusters
@@ -82,12 +87,21 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t *__restrict__ c
   const int excl = warp_tot[w] + incl - total;
   if (c < C) {
     offsets[static_cast<size_t>(h) * (C + 1) + c] = excl;
-    for (int k = 0; k < nch; ++k) cc[static_cast<size_t>(k) * C + c] += excl;
+    for (int k0 = 0; k0 < nch; k0 += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = k0 + u < nch ? cc[static_cast<size_t>(k0 + u) * C + c] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (k0 + u < nch) cc[static_cast<size_t>(k0 + u) * C + c] = v[u] + excl;
+    }
   }
   if (c == 0) offsets[static_cast<size_t>(h) * (C + 1) + C] = N;
 }
 
 // One warp per chunk: stable ranks inside each 32-token group via match_any.
+// The chunk's ids are loaded up front (kChunk / 32 per lane), so the ordered
+// walk over the groups waits on no global load.
 __global__ void __launch_bounds__(32) sort_scatter_kernel(const int32_t *__restrict__ assign,
                                                           int N, int C,
                                                           const int32_t *__restrict__ chunk_base,
@@ -102,9 +116,18 @@ __global__ void __launch_bounds__(32) sort_scatter_kernel(const int32_t *__restr
   int32_t *p = perm + static_cast<size_t>(h) * N;
   const int n0 = chunk * kChunk, n1 = min(N, n0 + kChunk);
   const unsigned lt = (1u << lane) - 1u;
-  for (int g = n0; g < n1; g += 32) {
+  int ids[kChunk / 32];
+#pragma unroll
+  for (int gi = 0; gi < kChunk / 32; ++gi) {
+    const int n = n0 + gi * 32 + lane;
+    ids[gi] = n < n1 ? a[n] : -1;
+  }
+#pragma unroll
+  for (int gi = 0; gi < kChunk / 32; ++gi) {
+    const int g = n0 + gi * 32;
+    if (g >= n1) break;
     const int n = g + lane;
-    int c = (n < n1) ? a[n] : -1;
+    int c = ids[gi];
     const bool ok = (c >= 0 && c < C);
     const unsigned live = __ballot_sync(0xffffffffu, ok);
     const unsigned peers = __match_any_sync(0xffffffffu, ok ? c : -1) & live;

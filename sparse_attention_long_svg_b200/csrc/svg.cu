@@ -439,13 +439,19 @@ size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq) {
   return bytes;
 }
 
-svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
-                           const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
-                           const int32_t *sel_count, const int32_t *sel_cols, float scale,
-                           void *op, float *lse, void *ws, size_t ws_bytes,
-                           svg_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Shared body of svg_sparse_attn (perm == nullptr: permuted output rows) and
+// svg_sparse_attn_unpermuted (row r of a head stored at row perm[r]).
+svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
+                            const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
+                            const int32_t *sel_count, const int32_t *sel_cols, float scale,
+                            const int32_t *perm, void *op, float *lse, void *ws, size_t ws_bytes,
+                            svg_stream_t stream) {
   if (!qp || !kp || !vp || !q_off || !k_off || !sel_count || !sel_cols || !op || !ws)
     return SVG_ERR_INVALID_ARG;
+  if (perm != nullptr && (op == qp || op == kp || op == vp)) return SVG_ERR_INVALID_ARG;
   if (!sizes_ok(BH, N) || Cq < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
   if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16) ||
@@ -481,6 +487,7 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
   prm.num_items = w.num_items;
   prm.op = static_cast<__nv_bfloat16 *>(op);
   prm.lse = lse;
+  prm.perm = perm;
   prm.N = N;
   prm.Cq = Cq;
   prm.Ck = Ck;
@@ -501,7 +508,30 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
     sparse_attn_kernel<64><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
   }
   if (pe) cudaEventRecord(pe[1], s);
-  return launch_status();
+  return launch_status("sparse_attn_kernel");
+}
+}  // namespace
+
+extern "C" {
+
+svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
+                           const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
+                           const int32_t *sel_count, const int32_t *sel_cols, float scale,
+                           void *op, float *lse, void *ws, size_t ws_bytes,
+                           svg_stream_t stream) {
+  return sparse_attn_impl(qp, kp, vp, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale,
+                          nullptr, op, lse, ws, ws_bytes, stream);
+}
+
+svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void *vp, int BH,
+                                      int N, int D, const int32_t *q_off, int Cq,
+                                      const int32_t *k_off, int Ck, const int32_t *sel_count,
+                                      const int32_t *sel_cols, float scale, const int32_t *perm_q,
+                                      void *o, float *lse, void *ws, size_t ws_bytes,
+                                      svg_stream_t stream) {
+  if (!perm_q) return SVG_ERR_INVALID_ARG;
+  return sparse_attn_impl(qp, kp, vp, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale,
+                          perm_q, o, lse, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -202,6 +202,30 @@ def test_sparse_attention_matches_oracle(name, case_data):
         assert np.max(np.abs(got_lse[h] - want_lse)) < 1e-3
 
 
+@pytest.mark.parametrize("name", list(CASES))
+def test_fused_unpermute_equals_separate_pass(name, case_data):
+    """svg_sparse_attn_unpermuted == svg_sparse_attn then svg_unpermute, bit for bit (lse too)."""
+    L, ref = case_data(name)
+    qp, kp, vp, q_off, k_off, op, lse = run_attention_from_oracle(L, ref)
+    perm = dev_i32(np.stack([r.perm_q for r in ref]))
+    want = svg.unpermute(op, perm)
+    H, N, D = L.q.shape
+    cnt = np.zeros((H, q_off.shape[1] - 1), np.int32)
+    cols = np.full((H, q_off.shape[1] - 1, k_off.shape[1] - 1), -1, np.int32)
+    for h in range(H):
+        for i, s in enumerate(ref[h].selection):
+            cnt[h, i] = len(s.cols)
+            cols[h, i, :len(s.cols)] = s.cols
+    o, lse_o = svg.sparse_attn(dev_bf16(qp), dev_bf16(kp), dev_bf16(vp), dev_i32(q_off), dev_i32(k_off),
+                               dev_i32(cnt), dev_i32(cols), want_lse=True, perm_q=perm)
+    torch.cuda.synchronize()
+    assert svg.get_error() == 0
+    assert torch.equal(o, want)
+    lse_want = torch.empty_like(lse)
+    lse_want.scatter_(1, perm.long(), lse)
+    assert torch.equal(lse_o, lse_want)
+
+
 def test_sparse_attention_all_blocks_equals_dense(case_data):
     L, ref = case_data("tiny")
     H, N, D = L.q.shape
