@@ -105,6 +105,13 @@ class ClockSampler:
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return self
+        # the sampler must already be streaming when the timed region starts
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
@@ -398,7 +405,7 @@ def run_svg(args, wl):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nh = 2
+        nh = 8                     # about 10 s of CPU work on the GPU machine's host
         secs, fl = oracle_sample(wl, nh)
         cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{nh} of {wl.heads} heads of the {wl.name} layer, whole path, {secs:.1f} s"}
@@ -436,7 +443,7 @@ def load_traffic(kernel: str, workload: str):
     if not entry:
         return None
     from sparse_attention_long_svg_b200 import build
-    if entry.get("source_hash") != build.source_hash():
+    if entry.get("source_hash") != build.source_hash(kernel):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -444,7 +451,7 @@ def load_traffic(kernel: str, workload: str):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="480p-5s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svg", choices=["svg", "reference"])

@@ -28,11 +28,24 @@ def sources():
     return sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
 
 
-def source_hash() -> str:
-    """Hash of every CUDA source and the ABI header (identifies a kernel build)."""
+# The source files each profiled kernel is compiled from (its own header and
+# the shared primitives); a profile's counters stay valid while these match.
+KERNEL_SOURCES = {
+    "kmeans_assign_tc_kernel": ("common.cuh", "kmeans_tc.cuh"),
+    "sparse_attn_kernel": ("common.cuh", "attn.cuh"),
+}
+
+
+def source_hash(kernel: str | None = None) -> str:
+    """Hash of the CUDA sources and the ABI header (a whole build), or of the
+    files one kernel in KERNEL_SOURCES is compiled from."""
     import hashlib
     h = hashlib.sha256()
-    for path in sources() + [os.path.join(os.path.dirname(HERE), "include", "svg.h")]:
+    if kernel is None:
+        paths = sources() + [os.path.join(os.path.dirname(HERE), "include", "svg.h")]
+    else:
+        paths = [os.path.join(HERE, "csrc", f) for f in KERNEL_SOURCES[kernel]]
+    for path in paths:
         with open(path, "rb") as f:
             h.update(os.path.basename(path).encode())
             h.update(f.read())

@@ -20,7 +20,9 @@
 //   warp 8     TMA producer: Q tiles, K and V boxes into 3-stage rings
 //   warp 9     MMA issuer: S_x = Q_x K^T into TMEM (two buffers per tile) and
 //              O_x += P_x V into TMEM, issuing whichever is ready; owns TMEM
-//   warp 10    item loader: the next item's key ranges into shared memory
+//   warp 10    item loader: claims the next item of the cost-sorted list from a
+//              counter shared by all CTAs and puts its header and key ranges
+//              into a 2-slot ring that every other role reads
 // P is written by the softmax warps to shared memory (bf16, 128-byte
 // swizzled, K-major) so both MMAs read their operands from shared memory.
 // O accumulates in TMEM across the item's key tiles; the softmax warps
@@ -35,9 +37,13 @@ namespace svg {
 constexpr int kItemRows = 256;     // query rows per work item (two 128-row tiles)
 constexpr int kSlotsPerTile = 8;   // 8-row slots per 64-key tile
 
-struct AttnItem {  // up to 256 query rows of one q-cluster
+struct AttnItem {  // up to 256 query rows of one q-cluster; h < 0 ends the list
   int32_t h, i, q0, packed;  // packed = rows (<= 256) | key_tiles << 9
 };
+
+// Readers of an item slot that must release it before it is refilled: the
+// producer, the MMA issuer and the eight softmax warps.
+constexpr int kItemReaders = 10;
 
 template <int D>
 struct AttnCfg {
@@ -108,6 +114,7 @@ struct AttnParams {
   const int32_t *q_off, *k_off, *sel_count, *sel_cols;
   const AttnItem *items;
   const int32_t *num_items;
+  int32_t *next_item;    // work counter: CTAs claim items in list order (zero at launch)
   __nv_bfloat16 *op;
   float *lse;
   const int32_t *perm;   // optional: write row r of a head to row perm[r] (un-permuted output)
@@ -180,7 +187,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       mbar_init(&B->p_full[x], 4);
       mbar_init(&B->o_full[x], 1);
       mbar_init(&B->item_full[x], 1);
-      mbar_init(&B->item_empty[x], 1);
+      mbar_init(&B->item_empty[x], kItemReaders);
     }
     mbar_init(&B->drain, 1);
     B->abort_flag = 0;
@@ -203,17 +210,30 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   const uint32_t tmem = B->tmem_base;
   const int total = *P.num_items;
   const uint64_t ns = P.wait_ns;
-  const int grid = static_cast<int>(gridDim.x);
 
   if (warp == Cfg::LOADER_WARP) {
     // ------------------------------------------------------------ item loader
-    int n = 0;
-    for (int w = blockIdx.x; w < total; w += grid, ++n) {
+    // Claims the next item of the list (longest first) with an atomic counter,
+    // so an SM that finishes early takes more work; after the last item it
+    // publishes an end marker (h = -1).
+    for (int n = 0;; ++n) {
       const int buf = n & 1;
       bool ok = true;
       if (lane == 0 && n >= 2)
         ok = attn_wait(B, &B->item_empty[buf], ((n >> 1) - 1) & 1, ns, SITE_ATTN_PRODUCER);
       if (!__shfl_sync(0xffffffffu, ok, 0) || warp_aborted(B)) break;
+      int w = 0;
+      if (lane == 0) w = atomicAdd(P.next_item, 1);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (w >= total) {
+        if (lane == 0) {
+          B->item[buf] = AttnItem{-1, 0, 0, 0};
+          B->item_cnt[buf] = 0;
+          __threadfence_block();
+          mbar_arrive(&B->item_full[buf]);
+        }
+        break;
+      }
       const AttnItem it = P.items[w];
       const int cnt = min(P.sel_count[it.h * P.Cq + it.i], Cfg::MAX_SEL);
       const int32_t *cols = P.sel_cols + static_cast<size_t>(it.h * P.Cq + it.i) * P.Ck;
@@ -255,10 +275,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     int n_items = 0;
     if (lane == 0) {
       bool ok = true;
-      for (int w = blockIdx.x; w < total && ok && !aborted(B); w += grid, ++n_items) {
+      for (; ok && !aborted(B); ++n_items) {
         const int buf = n_items & 1;
         if (!attn_wait(B, &B->item_full[buf], (n_items >> 1) & 1, ns, SITE_ATTN_PRODUCER)) break;
         const AttnItem it = B->item[buf];
+        if (it.h < 0) {                     // end of the list
+          mbar_arrive(&B->item_empty[buf]);
+          break;
+        }
         const int cnt = B->item_cnt[buf];
         const int2 *ranges = sRanges + buf * Cfg::MAX_SEL;
         const int ntk = it.packed >> 9;
@@ -354,24 +378,43 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     // Two cursors walk this CTA's key tiles: gs = next tile for S, gp = next
     // tile for PV; each tile has one S (and one PV) per query tile present.
     // Every pass issues whatever is ready (S first), so neither waits behind
-    // the other's operands.
+    // the other's operands.  The S cursor takes item headers from the item
+    // ring and queues them (hq) for the PV cursor, which trails it by up to
+    // two items.
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV),
                      p_base = smem_u32(sP);
-      int ws = blockIdx.x, wp = blockIdx.x, n_s = 0;
+      uint32_t n_hdr = 0, n_s = 0, n_pd = 0;   // headers read, items with all S / all PV issued
+      int hq[4] = {0, 0, 0, 0};
+      bool s_active = false, s_end = false;
       int ts = 0, tp = 0;
-      int pk_s = ws < total ? P.items[ws].packed : 0;
-      int pk_p = pk_s;
-      int pk_next = ws + grid < total ? P.items[ws + grid].packed : 0;
+      int pk_s = 0;
       uint32_t gs = 0, gp = 0;
       uint32_t n_sx[2] = {0, 0}, n_px[2] = {0, 0};
       bool s_done[2] = {false, false}, p_done[2] = {false, false};
       bool q_ok = false;
       const long long limit = static_cast<long long>(ns) * 2;
       long long t_last = clock64();
-      while (wp < total) {
+      while (true) {
         bool progress = false;
-        if (ws < total) {
+        if (!s_active && !s_end &&
+            mbar_test(&B->item_full[n_hdr & 1], (n_hdr >> 1) & 1)) {   // next item for the S cursor
+          const AttnItem it = B->item[n_hdr & 1];
+          mbar_arrive(&B->item_empty[n_hdr & 1]);
+          ++n_hdr;
+          if (it.h < 0) {
+            s_end = true;
+          } else {
+            pk_s = it.packed;
+            hq[n_s & 3] = pk_s;
+            s_active = true;
+            ts = 0;
+            q_ok = false;
+          }
+          progress = true;
+        }
+        if (s_end && !s_active && n_pd == n_s) break;   // every started item is finished
+        if (s_active) {
           const int ks = static_cast<int>(gs % 3);
           const bool has_b = (pk_s & 0x1FF) > Cfg::BM;
           if (!q_ok) q_ok = mbar_test(&B->q_full, n_s & 1);
@@ -400,12 +443,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               mma_commit(&B->k_empty[ks]);
               if (++ts == (pk_s >> 9)) {         // last S of this item: Q may be replaced
                 mma_commit(&B->q_empty);
-                ws += grid;
                 ++n_s;
-                ts = 0;
-                pk_s = pk_next;
-                pk_next = ws + grid < total ? P.items[ws + grid].packed : 0;
-                q_ok = false;
+                s_active = false;
               }
               ++gs;
               s_done[0] = s_done[1] = false;
@@ -413,6 +452,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
         if (gp < gs) {
+          const int pk_p = hq[n_pd & 3];
           const int vs = static_cast<int>(gp % 3);
           const bool has_b = (pk_p & 0x1FF) > Cfg::BM;
           if (mbar_test(&B->v_full[vs], (gp / 3) & 1)) {
@@ -437,9 +477,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             if (p_done[0] && (p_done[1] || !has_b)) {
               mma_commit(&B->v_empty[vs]);
               if (++tp == (pk_p >> 9)) {
-                wp += grid;
+                ++n_pd;
                 tp = 0;
-                pk_p = wp < total ? P.items[wp].packed : 0;
               }
               ++gp;
               p_done[0] = p_done[1] = false;
@@ -475,10 +514,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     uint8_t *sPx = sP + x * Cfg::P_BYTES;
     const float sl2 = P.scale_log2;
     uint32_t g = 0, n_s = 0, n_o = 0;
-    AttnItem next_it = blockIdx.x < total ? P.items[blockIdx.x] : AttnItem{0, 0, 0, 0};
-    for (int w = blockIdx.x; w < total && !warp_aborted(B); w += grid) {
-      const AttnItem it = next_it;
-      if (w + grid < total) next_it = P.items[w + grid];  // prefetch
+    for (uint32_t n = 0; !warp_aborted(B); ++n) {
+      if (!attn_warp_wait(B, &B->item_full[n & 1], (n >> 1) & 1, ns, SITE_ATTN_SOFTMAX)) break;
+      const AttnItem it = B->item[n & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B->item_empty[n & 1]);
+      if (it.h < 0) break;                  // end of the list
       const int ntk = it.packed >> 9;
       const int rows_total = it.packed & 0x1FF;
       const int nrows = x == 0 ? min(rows_total, Cfg::BM) : rows_total - Cfg::BM;
@@ -660,29 +701,37 @@ __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
   ktiles[idx] = (slots + kSlotsPerTile - 1) / kSlotsPerTile;
 }
 
-// Single block: one AttnItem per 256 query rows, ordered for the persistent kernel.
-// Items are sorted by key-tile count, longest first (a counting sort over
-// kAttnBuckets buckets), and the sorted list is laid out in "snake" order:
-// rank r goes to round k = r / grid, slot j = r % grid, reversed on odd
-// rounds.  The attention kernel gives CTA b the items b, b + grid, ..., so
-// every CTA gets one item of each round and the rounds alternate direction,
-// which evens out the work per SM (longest-processing-time-first).
+// Single block: one AttnItem per 256 query rows, in descending order of
+// estimated cost (key tiles x query tiles of the item; a counting sort over
+// kAttnBuckets buckets).  The attention kernel's CTAs claim items in this
+// order from a shared counter (greedy list scheduling, longest first), so an
+// SM that drew short items takes more of them.  Also resets that counter.
 constexpr int kAttnBuckets = 1024;
+
+__device__ __forceinline__ int attn_item_bucket(int kt, int rows) {
+  const int cost = kt * (rows > 128 ? 2 : 1);
+  return kAttnBuckets - 1 - min(cost, kAttnBuckets - 1);   // descending cost
+}
 
 __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
     const int32_t *__restrict__ q_off, const int32_t *__restrict__ qtiles,
-    const int32_t *__restrict__ ktiles, int BH, int Cq, int grid, AttnItem *__restrict__ items,
-    int32_t *__restrict__ num_items) {
+    const int32_t *__restrict__ ktiles, int BH, int Cq, AttnItem *__restrict__ items,
+    int32_t *__restrict__ num_items, int32_t *__restrict__ next_item) {
   __shared__ int hist[kAttnBuckets];
   __shared__ int warp_tot[32];
   const int total = BH * Cq;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   hist[threadIdx.x] = 0;
+  if (threadIdx.x == 0) *next_item = 0;
   __syncthreads();
-  // bucket b = kAttnBuckets - 1 - min(kt, kAttnBuckets - 1): descending cost
   for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int v = qtiles[idx];
-    if (v > 0) atomicAdd(&hist[kAttnBuckets - 1 - min(ktiles[idx], kAttnBuckets - 1)], v);
+    const int qt = qtiles[idx];
+    if (qt <= 0) continue;
+    const int kt = ktiles[idx];
+    const int h = idx / Cq, i = idx % Cq;
+    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_off[h * (Cq + 1) + i + 1];
+    for (int t = 0; t < qt; ++t)
+      atomicAdd(&hist[attn_item_bucket(kt, min(kItemRows, row1 - row0 - t * kItemRows))], 1);
   }
   __syncthreads();
   // exclusive scan of the buckets (one per thread)
@@ -709,26 +758,19 @@ __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
   const int excl = warp_tot[w] + incl - v;
   __syncthreads();
   hist[threadIdx.x] = excl;                       // now: next free rank of each bucket
-  if (threadIdx.x == kAttnBuckets - 1) {
-    *num_items = excl + v;
-    warp_tot[0] = excl + v;
-  }
+  if (threadIdx.x == kAttnBuckets - 1) *num_items = excl + v;
   __syncthreads();
-  const int n_items = warp_tot[0];
   for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
     const int qt = qtiles[idx];
     if (qt <= 0) continue;
     const int kt = ktiles[idx];
-    const int r0 = atomicAdd(&hist[kAttnBuckets - 1 - min(kt, kAttnBuckets - 1)], qt);
     const int h = idx / Cq, i = idx % Cq;
     const int row0 = q_off[h * (Cq + 1) + i], row1 = q_off[h * (Cq + 1) + i + 1];
     for (int t = 0; t < qt; ++t) {
-      const int rank = r0 + t;
-      const int round = rank / grid, slot = rank % grid;
-      const int in_round = min(grid, n_items - round * grid);   // the last round may be partial
-      const int pos = round * grid + ((round & 1) ? in_round - 1 - slot : slot);
       const int q0 = row0 + t * kItemRows;
-      items[pos] = AttnItem{h, i, q0, min(kItemRows, row1 - q0) | (kt << 9)};
+      const int rows = min(kItemRows, row1 - q0);
+      const int rank = atomicAdd(&hist[attn_item_bucket(kt, rows)], 1);
+      items[rank] = AttnItem{h, i, q0, rows | (kt << 9)};
     }
   }
 }

@@ -137,13 +137,14 @@ KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
 }
 
 struct AttnWs {
-  int32_t *num_items, *qtiles, *ktiles;
+  int32_t *num_items, *next_item, *qtiles, *ktiles;
   AttnItem *items;
 };
 AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
   Carve c{static_cast<uint8_t *>(ws)};
   AttnWs w;
   w.num_items = c.take<int32_t>(1);
+  w.next_item = c.take<int32_t>(1);
   w.qtiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.ktiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + kItemRows - 1) / kItemRows + Cq));
@@ -466,8 +467,8 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   const int pairs = BH * Cq;
   attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
                                                             Cq, Ck, w.qtiles, w.ktiles);
-  attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, num_sms(),
-                                                   w.items, w.num_items);
+  attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, w.items,
+                                                   w.num_items, w.next_item);
   svg_status st = launch_status();
   if (st != SVG_OK) return st;
 
@@ -485,6 +486,7 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   prm.sel_cols = sel_cols;
   prm.items = w.items;
   prm.num_items = w.num_items;
+  prm.next_item = w.next_item;
   prm.op = static_cast<__nv_bfloat16 *>(op);
   prm.lse = lse;
   prm.perm = perm;
