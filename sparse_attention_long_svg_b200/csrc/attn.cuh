@@ -546,25 +546,24 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&B->s_free[x][sb]);   // S buffer may be overwritten now
         ++n_s;
-        // masked scaled scores (log2 domain) and tile max; the mask is warp-uniform
+        // masked raw scores and the tile max; the mask is warp-uniform.  The
+        // scale (into the log2 domain) is applied once to the max and folded
+        // into one FMA per probability below (scale > 0 keeps the order).
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (mk[c] == 0xFFFFFFFFu) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              sv[c][e] *= sl2;
-              mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
-            }
+            for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              sv[c][e] = ((mk[c] >> e) & 1u) ? sv[c][e] * sl2 : -INFINITY;
+              sv[c][e] = ((mk[c] >> e) & 1u) ? sv[c][e] : -INFINITY;
               mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
             }
           }
         }
-        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         float alpha = 1.f;
         if (mt > m_ref + kRescaleLog2) {   // also taken on the first tile (m_ref = -inf)
           alpha = ex2_approx(m_ref - mt);
@@ -577,8 +576,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(sv[c][e] - m_ref);
-            const float p1 = ex2_approx(sv[c][e + 1] - m_ref);
+            const float p0 = ex2_approx(fmaf(sv[c][e], sl2, -m_ref));
+            const float p1 = ex2_approx(fmaf(sv[c][e + 1], sl2, -m_ref));
             rs2[0] += p0;
             rs2[1] += p1;
             packed[c * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
