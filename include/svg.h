@@ -12,6 +12,9 @@
  *   svg_sparse_attn  section 2(c) "Customized attention kernel"
  *   svg_unpermute    section 2(a) "Mathematical equivalence"
  *
+ * svg_sparse_attn_unpermuted is the last two in one kernel (the
+ * un-permutation done by the attention kernel's store).
+ *
  * Conventions shared by every call
  * --------------------------------
  *  - Tensors are head-major: a [BH, N, D] tensor holds BH = batch*heads
@@ -234,8 +237,8 @@ void svg_debug_set_fault(int fault);
  * Live per-kernel timing for benchmarks.  While enabled, the library records
  * a pair of CUDA events on the caller's stream around every launch of its two
  * heavy kernels: kernel 0 = the k-means assign kernel (inside svg_kmeans),
- * kernel 1 = the block-sparse attention kernel (inside svg_sparse_attn,
- * without its planning kernels).  Events come from a fixed pool created on
+ * kernel 1 = the block-sparse attention kernel (inside svg_sparse_attn and
+ * svg_sparse_attn_unpermuted, without their planning kernels).  Events come from a fixed pool created on
  * the first enable (up to 1024 launches between reads; later launches are not
  * timed and are reported in `dropped`).  svg_profile_read waits for the
  * recorded events, returns the summed milliseconds and the number of timed
@@ -244,7 +247,7 @@ void svg_debug_set_fault(int fault);
 svg_status svg_profile_enable(int on);
 svg_status svg_profile_read(int kernel, double *ms, int *launches, int *dropped);
 
-/* Library version, e.g. "svg-b200 0.1 (sm_100a)". */
+/* Library version, e.g. "svg-b200 0.2 (sm_100a)". */
 const char *svg_version(void);
 
 #ifdef __cplusplus

@@ -269,7 +269,7 @@ const char *svg_last_cuda_error(void) {
   return copy;
 }
 
-const char *svg_version(void) { return "svg-b200 0.1 (sm_100a)"; }
+const char *svg_version(void) { return "svg-b200 0.2 (sm_100a)"; }
 
 void svg_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs; }
 
