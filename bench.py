@@ -199,20 +199,25 @@ def run_reference(args, wl):
     return 0
 
 
-def workload_config(wl, n_gpus, heads=None):
+def workload_config(wl, n_gpus, heads=None, iters=None, top_p=None):
     heads = heads or wl.heads
-    return {"workload": wl.name, "heads": heads, "tokens": wl.tokens, "grid": list(wl.grid),
-            "head_dim": wl.head_dim, "cq": wl.cq, "ck": wl.ck, "kmeans_iters": wl.iters, "top_p": wl.top_p[0],
+    cfg = {"workload": wl.name, "heads": heads, "tokens": wl.tokens, "grid": list(wl.grid),
+           "head_dim": wl.head_dim, "cq": wl.cq, "ck": wl.ck, "kmeans_iters": iters or wl.iters,
+           "top_p": top_p if top_p is not None else wl.top_p[0],
             "layers_per_step_per_gpu": 1, "parallelism": f"dp{n_gpus} (independent layers per GPU)",
             "l2": "inputs larger than L2 (Q/K/V bf16 = %.0f MB > 126 MB); no flush" %
                   (3 * heads * wl.tokens * wl.head_dim * 2 / 1e6)}
+    if wl.warm_iters:
+        cfg["warm_start"] = ("timed call 1 starts from call 0's final centroids (the centroid cache) "
+                             "and runs %d rounds" % wl.warm_iters)
+    return cfg
 
 
 # ----------------------------------------------------------------------------- GPU leg
 
-def kernel_launches_per_step(wl) -> int:
+def kernel_launches_per_step(iters: int) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
-    per_kmeans = 2 + 4 * wl.iters            # split, |x|^2 + T x (assign, refine, bucket, accumulate)
+    per_kmeans = 2 + 4 * iters               # split, |x|^2 + T x (assign, refine, bucket, accumulate)
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
     return 2 * per_kmeans + 2 * per_permute + 1 + 3       # select; plan x2 + attention (un-permute fused)
 
@@ -248,19 +253,33 @@ def run_svg(args, wl):
     svg.load_library()
     peaks, peak_kind = load_peaks()
 
-    L = synth.make_layer(wl, heads=args.heads)
-    BH, N, D = L.q.shape
-
     def to_dev(x):
         return torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(device)
 
+    p = args.top_p if args.top_p is not None else wl.top_p[0]
+    T = wl.warm_iters or wl.iters            # k-means rounds of the timed call
+    if wl.warm_iters:
+        # centroid cache: call 0 (cold, wl.iters rounds) on this step's predecessor,
+        # then the timed call 1 starts from its final centroids
+        L0 = synth.make_layer(wl, heads=args.heads, call=0)
+        BH, N, D = L0.q.shape
+        layer0 = svg.SvgLayer(BH, N, D, wl.cq, wl.ck, device)
+        cache_q = torch.from_numpy(L0.init_centroids("q")).to(device)
+        cache_k = torch.from_numpy(L0.init_centroids("k")).to(device)
+        layer0(to_dev(L0.q), to_dev(L0.k), to_dev(L0.v), cache_q, cache_k, wl.iters, p)
+        torch.cuda.synchronize()
+        del layer0, L0
+        L = synth.make_layer(wl, heads=args.heads, call=1)
+        mu_q0, mu_k0 = cache_q, cache_k
+    else:
+        L = synth.make_layer(wl, heads=args.heads)
+        mu_q0 = torch.from_numpy(L.init_centroids("q")).to(device)
+        mu_k0 = torch.from_numpy(L.init_centroids("k")).to(device)
+    BH, N, D = L.q.shape
     q, k, v = to_dev(L.q), to_dev(L.k), to_dev(L.v)
-    mu_q0 = torch.from_numpy(L.init_centroids("q")).to(device)
-    mu_k0 = torch.from_numpy(L.init_centroids("k")).to(device)
     mu_q, mu_k = mu_q0.clone(), mu_k0.clone()
     layer = svg.SvgLayer(BH, N, D, wl.cq, wl.ck, device)
     out = torch.empty_like(q)
-    p = wl.top_p[0]
     stream = torch.cuda.current_stream()
     stage_names = ["kmeans_q", "kmeans_k", "permute", "select", "attn+unpermute"]
 
@@ -269,10 +288,10 @@ def run_svg(args, wl):
         mu_k.copy_(mu_k0)
         if ev:
             ev[0].record()
-        svg.kmeans(q, mu_q, wl.iters, layer.assign_q, layer.n_q, layer.workspace)
+        svg.kmeans(q, mu_q, T, layer.assign_q, layer.n_q, layer.workspace)
         if ev:
             ev[1].record()
-        svg.kmeans(k, mu_k, wl.iters, layer.assign_k, layer.n_k, layer.workspace)
+        svg.kmeans(k, mu_k, T, layer.assign_k, layer.n_k, layer.workspace)
         if ev:
             ev[2].record()
         svg.permute(layer.assign_q, wl.cq, [q], [layer.qp], layer.perm_q, layer.q_off, layer.workspace)
@@ -350,7 +369,7 @@ def run_svg(args, wl):
         dv.copy_(hv, non_blocking=True)
         mu_q.copy_(hmq, non_blocking=True)
         mu_k.copy_(hmk, non_blocking=True)
-        o, _ = layer(dq, dk, dv, mu_q, mu_k, wl.iters, p, 0.0, out)
+        o, _ = layer(dq, dk, dv, mu_q, mu_k, T, p, 0.0, out)
         hout.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
@@ -372,7 +391,7 @@ def run_svg(args, wl):
                  "launch_ms": attn_kernel_ms, "launches": attn_n, "total_ms": attn_k_ms,
                  "algorithmic": "4*D*sum_selected(n_q*n_k) = %.4g FLOP per launch" % flops_layer}
     # assign launches alternate: iters on Q (C = cq) then iters on K (C = ck) per step
-    assign_flops = 2.0 * N * D * BH * wl.iters * (wl.cq + wl.ck) * args.steps
+    assign_flops = 2.0 * N * D * BH * T * (wl.cq + wl.ck) * args.steps
     assign_launch_ms = assign_ms / max(assign_n, 1)
     assign_tflops = assign_flops / (assign_ms * 1e-3) / 1e12 if assign_ms > 0 else 0.0
     roof_assign = {"kernel": f"kmeans_assign_tc_kernel<{D}>", "bound": "tensor", "achieved": assign_tflops,
@@ -386,8 +405,8 @@ def run_svg(args, wl):
     else:
         roofline, roofline_other = roof_attn, roof_assign
     tensor_bytes = BH * N * D * 2
-    km_flops = {c: 2.0 * N * c * D * BH * wl.iters for c in (wl.cq, wl.ck)}
-    km_bytes = 2.0 * tensor_bytes * wl.iters          # assign read + update read per round
+    km_flops = {c: 2.0 * N * c * D * BH * T for c in (wl.cq, wl.ck)}
+    km_bytes = 2.0 * tensor_bytes * T                 # assign read + update read per round
     stages = {
         "kmeans_q": {"ms": stage_ms["kmeans_q"], "tflops": km_flops[wl.cq] / stage_ms["kmeans_q"] / 1e9,
                      "gbs": km_bytes / stage_ms["kmeans_q"] / 1e6},
@@ -417,13 +436,13 @@ def run_svg(args, wl):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl, world, BH),
+            "config": workload_config(wl, world, BH, T, p),
             "attn_ms": stage_ms["attn+unpermute"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
             "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / e2e_steps},
-            "gpu_launches": kernel_launches_per_step(wl) * args.steps,
+            "gpu_launches": kernel_launches_per_step(T) * args.steps,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -456,6 +475,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="480p-5s", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="svg", choices=["svg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--top-p", type=float, default=None, help="override the workload's (first) top-p")
     ap.add_argument("--heads", type=int, default=None,
                     help="first H heads of the workload only (smaller case for profiler captures)")
     args = ap.parse_args(argv)
