@@ -552,16 +552,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          if (mk[c] == 0xFFFFFFFFu) {
+          if (mk[c] != 0xFFFFFFFFu) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              sv[c][e] = ((mk[c] >> e) & 1u) ? sv[c][e] : -INFINITY;
-              mx4[e & 3] = fmaxf(mx4[e & 3], sv[c][e]);
-            }
+            for (int e = 0; e < 32; ++e) sv[c][e] = ((mk[c] >> e) & 1u) ? sv[c][e] : -INFINITY;
           }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            mx4[(e >> 1) & 3] = max3f(mx4[(e >> 1) & 3], sv[c][e], sv[c][e + 1]);
         }
         const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         float alpha = 1.f;
@@ -570,17 +567,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           m_ref = mt;
         }
         // probabilities -> bf16 pairs, row sum
-        float rs2[2] = {0.f, 0.f};
+        // (pairs of scores go through one paired FMA and one paired add)
+        float2 rs2 = make_float2(0.f, 0.f);
         uint32_t packed[32];
+        const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(fmaf(sv[c][e], sl2, -m_ref));
-            const float p1 = ex2_approx(fmaf(sv[c][e + 1], sl2, -m_ref));
-            rs2[0] += p0;
-            rs2[1] += p1;
-            packed[c * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+            const float2 a2 = fma_f32x2(make_float2(sv[c][e], sv[c][e + 1]), sl2x2, nm2);
+            const float2 p2 = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+            rs2 = add_f32x2(rs2, p2);
+            packed[c * 16 + (e >> 1)] = pack_bf16x2(p2.x, p2.y);
           }
         }
         if (t >= 1) {  // PV_x(t-1) must be done before P_x and O_x are touched
@@ -599,7 +597,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             tmem_st_wait();
           }
         }
-        l = l * alpha + (rs2[0] + rs2[1]);
+        l = l * alpha + (rs2.x + rs2.y);
         // P row: 64 keys = one 128-byte swizzle row (K-major, 16-byte chunks ^ row % 8)
         uint8_t *prow = sPx + row * 128;
 #pragma unroll
