@@ -86,5 +86,15 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
     # attention: unsupported D, workspace too small
     assert lib.svg_sparse_attn(f, f, f, 1, 16, 80, f, 2, f, 2, f, f, 0.0, f, nul, f, 1 << 20, nul) == 2
     assert lib.svg_sparse_attn(f, f, f, 1, 4096, 64, f, 2, f, 2, f, f, 0.0, f, nul, f, 8, nul) == 3
+    # fused attention + un-permute: missing perm_q, output aliasing an input, small workspace
+    g = _p(FAKE + 4096)
+    assert lib.svg_sparse_attn_unpermuted(f, f, f, 1, 16, 64, f, 2, f, 2, f, f, 0.0, nul, g, nul, f,
+                                          1 << 20, nul) == 1
+    assert lib.svg_sparse_attn_unpermuted(f, g, g, 1, 16, 64, f, 2, f, 2, f, f, 0.0, g, f, nul, g,
+                                          1 << 20, nul) == 1
+    assert lib.svg_sparse_attn_unpermuted(f, f, f, 1, 4096, 64, f, 2, f, 2, f, f, 0.0, f, g, nul, f,
+                                          8, nul) == 3
     # unpermute: aliasing
     assert lib.svg_unpermute(f, f, 1, 16, 64, f, nul) == 1
+    # nothing above reached CUDA
+    assert lib.svg_last_cuda_error().decode() == ""
