@@ -21,7 +21,7 @@ Semantic-Aware Permutation" (technical summary, section 2 "Methodology"):
       denoising step's centroids; "Customized attention kernel": attention
       over variable-size (q-cluster, k-cluster) blocks.
 
-Readings taken where the page is silent (each is listed in the design doc):
+Readings taken where the page is silent:
   * k-means uses squared Euclidean distance; ties go to the lowest cluster
     index; an empty cluster keeps its previous centroid; the returned
     assignment is the one of the last assign step and the returned centroids
