@@ -167,59 +167,103 @@ def centroid_weights(mu_q_i: np.ndarray, mu_k: np.ndarray, n_k: np.ndarray, scal
     return w / w.sum()
 
 
+# Unit roundoff of float64.
+U64 = 2.0 ** -53
+# Two weights closer than this (relative) are treated as equal at the cut: a
+# float64 evaluation of either weight may order them either way.
+TIE_REL = 2.0 ** -38
+
+
+def selection_band(mu_q_i: np.ndarray, mu_k: np.ndarray, n_k: np.ndarray, scale: float) -> float:
+    """How far two float64 evaluations of one row's normalised prefix masses can differ.
+
+    The top-p cut of a row is a comparison of prefix masses with p; both this
+    oracle and a float64 kernel evaluate them with rounding.  Bound (standard
+    forward error analysis, u = 2^-53, gamma_n = n u / (1 - n u)):
+      * logit_j = scale * mu_q . mu_k_j over D channels: error at most
+        scale * gamma_D * sum_d |mu_q_d mu_k_jd| + u |logit_j|; the row max
+        shifts by at most the same amount;
+      * a weight n_j exp(logit_j - max) then carries a relative error
+        rho <= 2 * max_j (logit error) + 4u (exp and the product);
+      * a normalised prefix C_k / S moves by at most 2 rho from the weights
+        plus 2 gamma_(n + 8) from the two sums over n live clusters, and the
+        threshold p * S by u.
+    The band covers both evaluations (twice one evaluation's bound).
+    """
+    mu_q_i = np.asarray(mu_q_i, np.float64)
+    mu_k = np.asarray(mu_k, np.float64)
+    live = np.asarray(n_k) > 0
+    if not live.any():
+        return 0.0
+    D = mu_q_i.shape[0]
+    gamma_d = D * U64 / (1.0 - D * U64)
+    absdot = np.abs(mu_k[live]) @ np.abs(mu_q_i)
+    logits = (mu_k[live] @ mu_q_i) * float(scale)
+    dl = float(scale) * gamma_d * float(absdot.max()) + U64 * float(np.abs(logits).max())
+    rho = 2.0 * dl + 4.0 * U64
+    n = int(live.sum())
+    gamma_n = (n + 8) * U64 / (1.0 - (n + 8) * U64)
+    return 2.0 * (2.0 * rho + 2.0 * gamma_n + U64)
+
+
 @dataclass
 class RowSelection:
     cols: np.ndarray          # selected k-cluster ids, ascending
     order: np.ndarray         # all live k-clusters by descending weight (ties: lower id)
     weights: np.ndarray       # normalised weights [Ck]
-    undecided: bool           # the cut sits within `tol` of a float32-visible boundary
+    undecided: bool           # the cut sits within `band` of p, or between near-equal weights
+    band: float = 0.0         # the band the row was judged with
 
 
-def select_row(weights: np.ndarray, p: float, tol: float = 1e-4,
+def select_row(weights: np.ndarray, p: float, tol: float,
                live_mask: Optional[np.ndarray] = None) -> RowSelection:
     """Smallest prefix of the descending-score order whose mass reaches p.
 
     ``live_mask`` marks the non-empty k-clusters (default: weight > 0).
+    ``tol`` is the row's rounding band (``selection_band``): the row is marked
+    undecided when a prefix mass next to the cut lies within ``tol`` of p, or
+    when the last kept and the first dropped weights are equal within TIE_REL.
     """
     w = np.asarray(weights, np.float64)
     live = np.nonzero(w > 0 if live_mask is None else np.asarray(live_mask))[0]
     if len(live) == 0:
-        return RowSelection(np.zeros(0, np.int64), live, w, False)
+        return RowSelection(np.zeros(0, np.int64), live, w, False, tol)
     # descending weight, ties -> lower index (stable sort of ascending index list)
     order = live[np.argsort(-w[live], kind="stable")]
     if p >= 1.0:
-        return RowSelection(np.sort(order), order, w, False)
+        return RowSelection(np.sort(order), order, w, False, tol)
     csum = np.cumsum(w[order])
     k = int(np.searchsorted(csum, p, side="left")) + 1     # first prefix with csum >= p
     k = min(k, len(order))
     undecided = abs(csum[k - 1] - p) < tol or (k >= 2 and abs(csum[k - 2] - p) < tol)
     if k < len(order):
         wl, wn = w[order[k - 1]], w[order[k]]
-        undecided = undecided or (wl - wn) <= tol * wl
-    return RowSelection(np.sort(order[:k]), order, w, bool(undecided))
+        undecided = undecided or (wl - wn) <= TIE_REL * wl
+    return RowSelection(np.sort(order[:k]), order, w, bool(undecided), tol)
 
 
 def select_topp(mu_q: np.ndarray, n_q: np.ndarray, mu_k: np.ndarray, n_k: np.ndarray,
-                p: float, scale: float, tol: float = 1e-4) -> List[RowSelection]:
+                p: float, scale: float) -> List[RowSelection]:
     """Per q-cluster top-p block selection for one head.  Empty q-clusters select nothing."""
     rows = []
     for i in range(mu_q.shape[0]):
         if n_q[i] == 0:
             rows.append(RowSelection(np.zeros(0, np.int64), np.zeros(0, np.int64),
-                                     np.zeros(mu_k.shape[0]), False))
+                                     np.zeros(mu_k.shape[0]), False, 0.0))
             continue
-        rows.append(select_row(centroid_weights(mu_q[i], mu_k, n_k, scale), p, tol,
+        band = selection_band(mu_q[i], mu_k, n_k, scale)
+        rows.append(select_row(centroid_weights(mu_q[i], mu_k, n_k, scale), p, band,
                                np.asarray(n_k) > 0))
     return rows
 
 
-def selection_is_valid(gpu_cols: Sequence[int], weights: np.ndarray, p: float, tol: float = 1e-4) -> bool:
-    """Whether a selection is an acceptable minimal top-p set up to float32 rounding.
+def selection_is_valid(gpu_cols: Sequence[int], weights: np.ndarray, p: float, tol: float) -> bool:
+    """Whether a selection is an acceptable minimal top-p set up to rounding.
 
-    Accepts the set when (i) it only holds live clusters, (ii) every selected
-    weight is at least every unselected weight (within tol relative), (iii) its
-    mass reaches p - tol, and (iv) without its lightest member it stays
-    below p + tol.
+    ``tol`` is the row's band (``selection_band``).  Accepts the set when
+    (i) it only holds live clusters, (ii) every selected weight is at least
+    every unselected weight (within TIE_REL relative), (iii) its mass reaches
+    p - tol, and (iv) without its lightest member it stays below p + tol.
     """
     w = np.asarray(weights, np.float64)
     sel = np.asarray(sorted(set(int(c) for c in gpu_cols)), np.int64)
@@ -229,7 +273,7 @@ def selection_is_valid(gpu_cols: Sequence[int], weights: np.ndarray, p: float, t
     if p >= 1.0:
         return np.array_equal(sel, live)
     uns = np.setdiff1d(live, sel)
-    if len(uns) and w[sel].min() < w[uns].max() * (1 - tol):
+    if len(uns) and w[sel].min() < w[uns].max() * (1 - TIE_REL):
         return False
     mass = w[sel].sum()
     if mass < p - tol:

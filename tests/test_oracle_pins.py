@@ -46,6 +46,10 @@ def brute_softmax_row(q, keys, vals, scale):
     return out, m + math.log(tot)
 
 
+# Band used with hand-made weight vectors (a float64-sized rounding band).
+BAND = 1e-12
+
+
 def rnd(shape, seed, scale=1.0):
     return np.random.default_rng(seed).standard_normal(shape) * scale
 
@@ -118,6 +122,17 @@ def test_objective_non_increasing_tiny_workload():
             after = so.lloyd_objective(x, mu, a)     # update can only lower it
             assert after <= cur + 1e-9 * cur
             prev = after
+
+
+def test_lloyd_objective_matches_brute_force():
+    x, mu = rnd((23, 4), 24), rnd((5, 4), 25)
+    a = np.random.default_rng(26).integers(0, 5, 23)
+    brute = 0.0
+    for n in range(23):
+        for d in range(4):
+            diff = x[n, d] - mu[a[n], d]
+            brute += diff * diff
+    assert abs(so.lloyd_objective(x, mu, a) - brute) <= 1e-12 * brute
 
 
 def test_separated_mixture_recovers_regions():
@@ -201,7 +216,7 @@ def test_selection_reaches_p_and_is_minimal():
         w[rng.integers(0, 30, 3)] = 0
         w /= w.sum()
         p = float(rng.uniform(0.05, 0.99))
-        r = so.select_row(w, p)
+        r = so.select_row(w, p, BAND)
         sel = r.cols
         mass = w[sel].sum()
         assert mass >= p - 1e-12
@@ -209,7 +224,7 @@ def test_selection_reaches_p_and_is_minimal():
         uns = np.setdiff1d(np.nonzero(w > 0)[0], sel)
         if len(uns):
             assert w[sel].min() >= w[uns].max()          # exactly the top-|S|
-        assert so.selection_is_valid(sel, w, p)
+        assert so.selection_is_valid(sel, w, p, BAND)
 
 
 def test_p_one_keeps_every_live_cluster_and_empty_rows_select_nothing():
@@ -248,10 +263,65 @@ def test_one_token_per_cluster_is_token_level_top_p():
 
 def test_selection_validator_rejects_wrong_sets():
     w = np.array([0.5, 0.3, 0.15, 0.05])
-    assert so.selection_is_valid([0, 1], w, 0.75)
-    assert not so.selection_is_valid([0], w, 0.75)           # mass too small
-    assert not so.selection_is_valid([0, 1, 2], w, 0.75)     # not minimal
-    assert not so.selection_is_valid([0, 2], w, 0.6)         # skips a heavier cluster
+    assert so.selection_is_valid([0, 1], w, 0.75, BAND)
+    assert not so.selection_is_valid([0], w, 0.75, BAND)           # mass too small
+    assert not so.selection_is_valid([0, 1, 2], w, 0.75, BAND)     # not minimal
+    assert not so.selection_is_valid([0, 2], w, 0.6, BAND)         # skips a heavier cluster
+    # a cut one cluster short is rejected even when its mass misses p by only 1e-9
+    w2 = np.array([0.5, 0.4 - 1e-9, 0.1 + 1e-9])
+    assert not so.selection_is_valid([0, 1], w2, 0.9, BAND)
+    assert so.selection_is_valid([0, 1, 2], w2, 0.9, BAND)
+
+
+def _exact_prefix_masses(mu_q_i, mu_k, n_k, scale, order):
+    """Normalised prefix masses along `order`, from exact rational logits and 50-digit exp."""
+    from decimal import Decimal, localcontext
+    from fractions import Fraction
+    with localcontext() as ctx:
+        ctx.prec = 50
+        sc = Fraction(scale)
+        logits = {}
+        for j in range(len(n_k)):
+            if n_k[j] > 0:
+                dot = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(mu_q_i, mu_k[j]))
+                f = dot * sc
+                logits[j] = Decimal(f.numerator) / Decimal(f.denominator)
+        m = max(logits.values())
+        w = {j: Decimal(int(n_k[j])) * (logits[j] - m).exp() for j in logits}
+        tot = sum(w.values())
+        out, acc = [], Decimal(0)
+        for j in order:
+            acc += w[j]
+            out.append(float(acc / tot))
+        return np.array(out)
+
+
+def test_selection_band_bounds_the_float64_error():
+    """The band (twice one evaluation's bound) covers the oracle's own float64
+    prefix masses against 50-digit arithmetic, on rows with large centroids."""
+    rng = np.random.default_rng(31)
+    for trial in range(12):
+        D = (64, 128)[trial % 2]
+        C = int(rng.integers(20, 120))
+        mag = (1.0, 4.0, 12.0)[trial % 3]
+        mu_q = (rng.standard_normal(D) * mag).astype(np.float32).astype(np.float64)
+        mu_k = (rng.standard_normal((C, D)) * mag).astype(np.float32).astype(np.float64)
+        n_k = rng.integers(0, 90, C)
+        n_k[0] = 5
+        scale = 1.0 / math.sqrt(D)
+        band = so.selection_band(mu_q, mu_k, n_k, scale)
+        assert 0 < band < 1e-9                   # float64-sized, not a float32-sized band
+        w = so.centroid_weights(mu_q, mu_k, n_k, scale)
+        r = so.select_row(w, 0.9, band, n_k > 0)
+        exact = _exact_prefix_masses(mu_q, mu_k, n_k, scale, r.order)
+        got = np.cumsum(w[r.order])
+        assert np.max(np.abs(got - exact)) <= band / 2, (trial, np.max(np.abs(got - exact)), band)
+
+
+def test_golden_density(golden):
+    g = golden["density"]
+    pairs, frac = so.density(np.array(g["q_off"]), np.array(g["k_off"]), g["selection"])
+    assert pairs == g["pairs"] and frac == g["fraction"]
 
 
 # ----------------------------------------------------------------- attention
@@ -350,8 +420,8 @@ def test_pins_catch_planted_mistakes(monkeypatch, golden):
     # 3. top-p cut one element late (cumsum > p instead of >= p)
     origr = so.select_row
 
-    def late(w, p, tol=1e-4):
-        r = origr(w, p, tol)
+    def late(w, p, tol, live_mask=None):
+        r = origr(w, p, tol, live_mask)
         if p < 1 and len(r.cols) < len(r.order):
             r.cols = np.sort(r.order[:len(r.cols) + 1])
         return r
@@ -364,5 +434,18 @@ def test_pins_catch_planted_mistakes(monkeypatch, golden):
     _expect_failure(test_attention_rows_match_brute_force)
     monkeypatch.setattr(so, "softmax_attention_rows", origa)
     # 5. un-permute applied as a second gather instead of a scatter
+    origs = so.scatter_rows
     monkeypatch.setattr(so, "scatter_rows", lambda xp, perm: np.asarray(xp)[perm])
     _expect_failure(test_permutation_invariants)
+    monkeypatch.setattr(so, "scatter_rows", origs)
+    # 6. objective with unsquared differences
+    monkeypatch.setattr(so, "lloyd_objective", lambda x, mu, a: float(np.sum(
+        np.abs(np.asarray(x, np.float64) - np.asarray(mu, np.float64)[a]))))
+    _expect_failure(test_lloyd_objective_matches_brute_force)
+    # 7. density counting k-cluster sizes only (q-cluster size dropped)
+    monkeypatch.setattr(so, "density", lambda qo, ko, sel: (
+        float(sum(np.diff(ko)[np.asarray(c, np.int64)].sum() for c in sel if len(c))), 0.0))
+    _expect_failure(test_golden_density, golden)
+    # 8. a float32-sized rounding band (u = 2^-24) would swallow decided cuts
+    monkeypatch.setattr(so, "U64", 2.0 ** -24)
+    _expect_failure(test_selection_band_bounds_the_float64_error)
