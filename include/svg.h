@@ -128,7 +128,11 @@ svg_status svg_permute(const int32_t *assign, int BH, int N, int C, int32_t *per
  *   sel_cols  [BH, Cq, Ck] int32  out: row (h,i) holds its selected k-cluster ids in
  *                                 ascending order in its first sel_count entries;
  *                                 the remaining entries are left untouched
- * Requires 0 < p, Ck <= 1024; scale <= 0 selects 1/sqrt(D).  All math fp32.
+ * Requires 0 < p, Ck <= 1024; scale <= 0 selects 1/sqrt(D) (formed in
+ * float64).  The cut turns weights into an integer set, so logits, weights
+ * and prefix masses are evaluated in float64 (products of fp32 centroid
+ * channels are exact there); a float64 evaluation can differ from the exact
+ * cut only when a prefix mass lies within about 1e-12 of p.
  */
 svg_status svg_select_topp(const float *mu_q, const int32_t *n_q, const float *mu_k,
                            const int32_t *n_k, int BH, int Cq, int Ck, int D, float p, float scale,
@@ -149,7 +153,9 @@ svg_status svg_select_topp(const float *mu_q, const int32_t *n_q, const float *m
  *                                sum_j exp(scale * q.k_j) per row
  * Rows of empty q-clusters do not exist; every other row is written.  A row
  * whose cluster selected no key is left untouched and flagged with
- * SVG_ERR_DEVICE_CHECK.  scale <= 0 selects 1/sqrt(D).
+ * SVG_ERR_DEVICE_CHECK, and so is a sel_count outside [0, Ck] (it is clamped
+ * before any block list entry is read).  Requires Ck <= 1024
+ * (SVG_ERR_UNSUPPORTED otherwise).  scale <= 0 selects 1/sqrt(D).
  */
 size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq);
 svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
@@ -246,6 +252,15 @@ void svg_debug_set_fault(int fault);
  * record.  Timing adds two event records per launch and nothing else. */
 svg_status svg_profile_enable(int on);
 svg_status svg_profile_read(int kernel, double *ms, int *launches, int *dropped);
+
+/* While profiling is enabled, every attention launch also counts the
+ * (128-row query tile, 128-key tile) pairs it issues tensor-core work for: one
+ * S = Q K^T chain and one O += P V chain each, i.e. 4 * 128 * 128 * D
+ * multiply-add FLOPs including masked padding rows and columns.  This call
+ * waits for the device, returns the count accumulated since the previous call
+ * and resets it.  Issued FLOPs against the selected blocks' FLOPs give the
+ * padding waste of the variable-size blocks. */
+svg_status svg_profile_attn_pairs(uint64_t *pairs);
 
 /* Library version, e.g. "svg-b200 0.2 (sm_100a)". */
 const char *svg_version(void);

@@ -52,6 +52,7 @@ SIGNATURES = {
     "svg_profile_enable": (_I, [_I]),
     "svg_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
                               ctypes.POINTER(ctypes.c_int)]),
+    "svg_profile_attn_pairs": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
 }
 
 PROFILE_KERNELS = {"kmeans_assign": 0, "sparse_attn": 1}
@@ -137,6 +138,16 @@ def profile_read(kernel: str) -> Tuple[float, int, int]:
     _check("svg_profile_read", load_library().svg_profile_read(PROFILE_KERNELS[kernel], ctypes.byref(ms),
                                                                ctypes.byref(n), ctypes.byref(dropped)))
     return ms.value, n.value, dropped.value
+
+
+def profile_attn_pairs() -> int:
+    """(query tile, key tile) pairs the attention kernel issued MMAs for since the last call."""
+    v = ctypes.c_uint64()
+    _check("svg_profile_attn_pairs", load_library().svg_profile_attn_pairs(ctypes.byref(v)))
+    return int(v.value)
+
+
+ATTN_TILE = 128   # query rows and keys per (query tile, key tile) pair
 
 
 # --------------------------------------------------------------------- stages

@@ -179,6 +179,15 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
       : "memory");
 }
 
+// Brings the box at (x, y) of a 2-D tensor map into L2 (no shared-memory
+// destination, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -443,6 +452,51 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | (1u << 10)                                // B format: bf16
          | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor kept as its two 32-bit halves.  The low
+// half holds the start address in 16-byte units (bits 0-13); shared-memory
+// addresses stay below 256 KB, so a byte offset k is added to it as k >> 4
+// without a carry.  Building descriptors once and adding compile-time
+// offsets keeps the issuing thread to about one integer add per operand per
+// MMA: a single thread issues every MMA of a CTA, and its instruction latency
+// (not the tensor pipe) limits short MMAs when descriptors are rebuilt each time.
+struct SmemDesc {
+  uint32_t lo, hi;
+};
+
+__device__ __forceinline__ SmemDesc make_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  const uint64_t d = smem_desc_sw128(addr, lbo, sbo);
+  return SmemDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+
+// D[tmem] (+)= A * B^T, kind::f16, descriptors given as halves plus 16-byte
+// offsets of the start address.
+__device__ __forceinline__ void mma_bf16_ss_off(uint32_t d_tmem, SmemDesc a, uint32_t a_off,
+                                                SmemDesc b, uint32_t b_off, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+      "mov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo + a_off), "r"(a.hi), "r"(b.lo + b_off), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// A chain of STEPS K16 MMAs into one accumulator.  The operands are
+// 128-byte-swizzled tiles whose K dimension is cut into 64-element halves:
+// K-step k starts at byte offset (k / 4) * X_HALF + (k % 4) * X_K from its
+// tile's descriptor.  Fully unrolled: the offsets are immediates.
+template <int STEPS, uint32_t A_HALF, uint32_t A_K, uint32_t B_HALF, uint32_t B_K>
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, SmemDesc a, SmemDesc b, uint32_t idesc,
+                                          uint32_t accumulate_first) {
+#pragma unroll
+  for (int k = 0; k < STEPS; ++k) {
+    const uint32_t ao = ((k >> 2) * A_HALF + (k & 3) * A_K) >> 4;
+    const uint32_t bo = ((k >> 2) * B_HALF + (k & 3) * B_K) >> 4;
+    mma_bf16_ss_off(d_tmem, a, ao, b, bo, idesc, k > 0 ? 1u : accumulate_first);
+  }
 }
 
 // Byte offset of element (row, col) inside a K-major, 128-byte-swizzled tile

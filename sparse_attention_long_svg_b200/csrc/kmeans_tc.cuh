@@ -11,45 +11,59 @@
 // epilogue also counts the members of every cluster (the refine step moves
 // the tokens it reassigns), which the update step (kmeans.cuh) starts from.
 //
-// Persistent: one CTA per SM walks units (head, 128-token tile) in
-// head-major order (the head's centroids stay hot in L2).  Warps 0-7:
-// epilogue in two groups of four (thread t of a group = token t of the tile
-// = TMEM lane t), taking alternate chunks; warp 8: TMA producer (x tiles,
-// centroid chunks and their squared norms); warp 9: MMA issuer and TMEM
-// owner.  x tiles (2-deep ring) and centroid chunks of 128 (hi and lo parts,
-// 2-deep ring) stream through shared memory; four TMEM accumulators (two per
-// epilogue group) let the MMAs run up to two chunks ahead of each group.
+// Data movement is the limit of this step: a 128-token tile of x is 32 KB
+// but one 128-centroid chunk (hi and lo parts) is 64 KB, and streaming every
+// chunk from L2 for every tile saturates L2-to-shared-memory bandwidth long
+// before the tensor cores.  So every CTA takes a contiguous range of
+// (head, 128-token tile) units and reuses centroids across tiles:
+//   * C <= 128 (one chunk, SINGLE): the chunk stays in shared memory while
+//     the CTA's units belong to the same head; only x streams (4-deep ring);
+//   * C > 128: consecutive tiles of one head are taken in pairs, and every
+//     chunk (hi and lo parts through a 4-deep ring) feeds both tiles' MMA
+//     chains before it is released, halving the centroid traffic per tile.
+// Warps 0-7: epilogue in two groups of four; group g owns tile g of every
+// pair (thread t of a group = token t of the tile = TMEM lane t) and keeps
+// the running best pair over all chunks of its tile, so the groups never
+// merge.  Warp 8: TMA producer.  Warp 9: MMA issuer and TMEM owner; each
+// (tile, chunk) is one chain of 2 x D/16 MMAs (hi then lo) into one of the
+// group's two TMEM accumulators.
 #pragma once
 #include "common.cuh"
 
 namespace svg {
 
-template <int D>
+constexpr int kKmChunk = 128;   // centroids per chunk (MMA N)
+
+template <int D, bool SINGLE>
 struct KmCfg {
-  static constexpr int BM = 128, NC = 128, DH = D / 64;
-  static constexpr int XST = 2, CST = 2;  // x tile ring, centroid chunk ring
+  static constexpr int BM = 128, NC = kKmChunk, DH = D / 64;
+  static constexpr int XST = SINGLE ? 4 : 2;   // x tile ring
+  static constexpr int CST = SINGLE ? 2 : 4;   // centroid part ring (a part = hi or lo of a chunk)
   static constexpr int X_BYTES = BM * D * 2, C_BYTES = NC * D * 2;
-  static constexpr int HALF = 128 * 128;  // one 64-channel half of a 128-row tile
+  static constexpr int HALF = 128 * 128;       // one 64-channel half of a 128-row tile
   static constexpr int OFF_X = 0;
-  static constexpr int OFF_C = OFF_X + XST * X_BYTES;          // stage: hi part then lo part
-  static constexpr int NST = 4, AST = 4;  // norms ring, TMEM accumulators
-  static constexpr int OFF_NORM = OFF_C + CST * 2 * C_BYTES;   // NST x NC fp32 squared norms
-  static constexpr int OFF_MERGE = OFF_NORM + NST * NC * 4;    // 2 x 128 x (best, arg, second, arg2)
-  static constexpr int OFF_BAR = OFF_MERGE + 2 * 128 * 16;
+  static constexpr int OFF_C = OFF_X + XST * X_BYTES;
+  static constexpr int OFF_BAR = OFF_C + CST * C_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+  static constexpr int AST = 4;                // TMEM accumulators, two per epilogue group
   static constexpr uint32_t TM_COLS = AST * NC;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NC, false, false);
-  static constexpr int EPI_WARPS = 8;                          // two groups of four
+  static constexpr int EPI_WARPS = 8;          // two groups of four
   static constexpr int THREADS = (EPI_WARPS + 2) * 32;
   static constexpr int PRODUCER_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
 };
 
 struct KmBarriers {
-  uint64_t x_full[2], x_empty[2], c_full[2], c_empty[2], acc_full[4], acc_empty[4];
-  uint64_t n_full[4], n_empty[4], merge_full[2], merge_empty[2], drain;
+  uint64_t x_full[4], x_empty[4], c_full[4], c_empty[4], acc_full[4], acc_empty[4], drain;
   uint32_t tmem_base;
   int32_t abort_flag;
 };
+
+// Tiles (1 or 2) of the pair of units starting at u: two when u + 1 is in the
+// CTA's range and in the same head.
+__device__ __forceinline__ int km_pair_tiles(int u, int u_end, int tiles) {
+  return (u + 1 < u_end && (u + 1) / tiles == u / tiles) ? 2 : 1;
+}
 
 // One near-tie token: flat token index (h * N + n) and its two candidates.
 struct KmTie {
@@ -99,8 +113,8 @@ __global__ void kmeans_split_kernel(const float *__restrict__ mu, int C, int Cpa
   if (lane == 0) norms[static_cast<size_t>(h) * Cpad + c] = c < C ? s : kPadNorm;
 }
 
-template <int D>
-__global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
+template <int D, bool SINGLE>
+__global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
     kmeans_assign_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                             const __grid_constant__ CUtensorMap map_hi,
                             const __grid_constant__ CUtensorMap map_lo, int BH, int N, int C,
@@ -108,33 +122,27 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
                             const float *__restrict__ xnorm, int32_t *__restrict__ assign,
                             int32_t *__restrict__ counts, KmTie *__restrict__ ties,
                             int32_t *__restrict__ num_ties, uint64_t wait_ns) {
-  using Cfg = KmCfg<D>;
+  using Cfg = KmCfg<D, SINGLE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   KmBarriers *B = reinterpret_cast<KmBarriers *>(smem + Cfg::OFF_BAR);
-  float *sNorm = reinterpret_cast<float *>(smem + Cfg::OFF_NORM);
-  float4 *sMerge = reinterpret_cast<float4 *>(smem + Cfg::OFF_MERGE);
   const int warp = static_cast<int>(warp_id()), lane = static_cast<int>(lane_id());
   const int tiles = (N + Cfg::BM - 1) / Cfg::BM;
-  const int units = BH * tiles;              // unit u = (head u / tiles, tile u % tiles)
   const int nchunks = Cpad / Cfg::NC;
-  const int grid = static_cast<int>(gridDim.x);
+  // this CTA's contiguous range of units u = (head u / tiles, tile u % tiles)
+  const long long units = static_cast<long long>(BH) * tiles;
+  const int u_begin = static_cast<int>(units * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&B->x_full[s], 1);
-      mbar_init(&B->x_empty[s], 1);          // released by the MMA commit after a unit
+      mbar_init(&B->x_empty[s], 1);          // released by an MMA commit
       mbar_init(&B->c_full[s], 1);
       mbar_init(&B->c_empty[s], 1);
-      mbar_init(&B->merge_full[s], 4);
-      mbar_init(&B->merge_empty[s], 4);
-    }
-    for (int s = 0; s < 4; ++s) {
       mbar_init(&B->acc_full[s], 1);
       mbar_init(&B->acc_empty[s], 4);        // the four warps of the group that read it
-      mbar_init(&B->n_full[s], 1);
-      mbar_init(&B->n_empty[s], 4);
     }
     mbar_init(&B->drain, 1);
     B->abort_flag = 0;
@@ -148,96 +156,140 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
+  auto x_slot = [&](uint32_t n) { return smem + Cfg::OFF_X + (n % Cfg::XST) * Cfg::X_BYTES; };
+  auto c_slot = [&](uint32_t n) { return smem + Cfg::OFF_C + (n % Cfg::CST) * Cfg::C_BYTES; };
 
   if (warp == Cfg::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t nu = 0, gc = 0, gn = 0;   // x tiles, centroid chunks and norm rows issued
+      uint32_t nx = 0, nc = 0;   // x tiles and centroid parts issued
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += grid, ++nu) {
-        const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
-        const int xs = nu & 1;
-        if (nu >= 2 && !km_wait(B, &B->x_empty[xs], ((nu >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA)) break;
-        mbar_arrive_expect_tx(&B->x_full[xs], Cfg::X_BYTES);
-        uint8_t *xd = smem + Cfg::OFF_X + xs * Cfg::X_BYTES;
+      int cur_h = -1;
+      auto load_x = [&](int u) {
+        const uint32_t s = nx % Cfg::XST;
+        if (nx >= static_cast<uint32_t>(Cfg::XST) &&
+            !km_wait(B, &B->x_empty[s], ((nx / Cfg::XST) - 1) & 1, wait_ns, SITE_KMEANS_MMA))
+          return false;
+        mbar_arrive_expect_tx(&B->x_full[s], Cfg::X_BYTES);
 #pragma unroll
         for (int dh = 0; dh < Cfg::DH; ++dh)
-          tma_load_2d(xd + dh * Cfg::HALF, &map_x, dh * 64, h * N + n0, &B->x_full[xs]);
-        for (int j = 0; j < nchunks; ++j, ++gc) {
-          const int cs = gc & 1, ns = gc & 3;
-          if (gc >= 2 && !km_wait(B, &B->c_empty[cs], ((gc >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&B->c_full[cs], 2 * Cfg::C_BYTES);
-          uint8_t *cd = smem + Cfg::OFF_C + cs * 2 * Cfg::C_BYTES;
-          const int crow = h * Cpad + j * Cfg::NC;
+          tma_load_2d(x_slot(nx) + dh * Cfg::HALF, &map_x, dh * 64, (u / tiles) * N + (u % tiles) * Cfg::BM,
+                      &B->x_full[s]);
+        ++nx;
+        return true;
+      };
+      // one centroid part (hi or lo) of chunk j of head h
+      auto load_part = [&](int h, int j, int part) {
+        const uint32_t s = nc % Cfg::CST;
+        if (nc >= static_cast<uint32_t>(Cfg::CST) &&
+            !km_wait(B, &B->c_empty[s], ((nc / Cfg::CST) - 1) & 1, wait_ns, SITE_KMEANS_MMA))
+          return false;
+        mbar_arrive_expect_tx(&B->c_full[s], Cfg::C_BYTES);
 #pragma unroll
-          for (int dh = 0; dh < Cfg::DH; ++dh) {
-            tma_load_2d(cd + dh * Cfg::HALF, &map_hi, dh * 64, crow, &B->c_full[cs]);
-            tma_load_2d(cd + Cfg::C_BYTES + dh * Cfg::HALF, &map_lo, dh * 64, crow, &B->c_full[cs]);
+        for (int dh = 0; dh < Cfg::DH; ++dh)
+          tma_load_2d(c_slot(nc) + dh * Cfg::HALF, part ? &map_lo : &map_hi, dh * 64, h * Cpad + j * Cfg::NC,
+                      &B->c_full[s]);
+        ++nc;
+        return true;
+      };
+      for (int u = u_begin; u < u_end && ok; ) {
+        const int nt = km_pair_tiles(u, u_end, tiles);
+        const int h = u / tiles;
+        if (SINGLE) {
+          if (h != cur_h) {          // new head: its chunk replaces the resident one
+            ok = load_part(h, 0, 0) && load_part(h, 0, 1);
+            cur_h = h;
           }
-          if (gc >= 4 && !km_wait(B, &B->n_empty[ns], ((gc >> 2) - 1) & 1, wait_ns, SITE_KMEANS_MMA)) {
-            ++gc;          // this chunk's centroid copies are in flight: the drain waits for them
-            ok = false;
-            break;
+          for (int t = 0; t < nt && ok; ++t) ok = load_x(u + t);
+        } else {
+          for (int j = 0; j < nchunks && ok; ++j) {
+            ok = load_part(h, j, 0) && load_part(h, j, 1);
+            if (j == 0)
+              for (int t = 0; t < nt && ok; ++t) ok = load_x(u + t);
           }
-          mbar_arrive_expect_tx(&B->n_full[ns], Cfg::NC * 4);
-          bulk_load(sNorm + ns * Cfg::NC, norms + static_cast<size_t>(crow), Cfg::NC * 4, &B->n_full[ns]);
-          ++gn;
         }
+        u += nt;
       }
       // drain: wait for the last issued copies of each ring slot
       if (*reinterpret_cast<volatile int32_t *>(&B->abort_flag)) {
-        for (uint32_t k = nu >= 2 ? nu - 2 : 0; k < nu; ++k)
-          mbar_wait(&B->x_full[k & 1], (k >> 1) & 1, 1000000000ull);
-        for (uint32_t k = gc >= 2 ? gc - 2 : 0; k < gc; ++k)
-          mbar_wait(&B->c_full[k & 1], (k >> 1) & 1, 1000000000ull);
-        for (uint32_t k = gn >= 4 ? gn - 4 : 0; k < gn; ++k)
-          mbar_wait(&B->n_full[k & 3], (k >> 2) & 1, 1000000000ull);
+        for (uint32_t k = nx >= static_cast<uint32_t>(Cfg::XST) ? nx - Cfg::XST : 0; k < nx; ++k)
+          mbar_wait(&B->x_full[k % Cfg::XST], (k / Cfg::XST) & 1, 1000000000ull);
+        for (uint32_t k = nc >= static_cast<uint32_t>(Cfg::CST) ? nc - Cfg::CST : 0; k < nc; ++k)
+          mbar_wait(&B->c_full[k % Cfg::CST], (k / Cfg::CST) & 1, 1000000000ull);
       }
     }
   } else if (warp == Cfg::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t nu = 0, gc = 0;
+      uint32_t nx = 0, nc = 0, kacc[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += grid, ++nu) {
-        const int xs = nu & 1;
-        if (!km_wait(B, &B->x_full[xs], (nu >> 1) & 1, wait_ns, SITE_KMEANS_MMA)) break;
-        const uint32_t xb = smem_u32(smem + Cfg::OFF_X + xs * Cfg::X_BYTES);
-        for (int j = 0; j < nchunks; ++j, ++gc) {
-          const int cs = gc & 1, ab = gc & 3;
-          if (!km_wait(B, &B->c_full[cs], (gc >> 1) & 1, wait_ns, SITE_KMEANS_MMA) ||
-              (gc >= 4 && !km_wait(B, &B->acc_empty[ab], ((gc >> 2) - 1) & 1, wait_ns, SITE_KMEANS_MMA))) {
+      int cur_h = -1;
+      // descriptors of x slot 0 and centroid slot 0, built once; a slot adds its offset
+      const SmemDesc xd0 = make_desc_sw128(smem_u32(smem + Cfg::OFF_X), 16, 1024);
+      const SmemDesc cd0 = make_desc_sw128(smem_u32(smem + Cfg::OFF_C), 16, 1024);
+      for (int u = u_begin; u < u_end && ok; ) {
+        const int nt = km_pair_tiles(u, u_end, tiles);
+        const int h = u / tiles;
+        if (SINGLE && h != cur_h) {   // the resident chunk of the previous head is no longer read
+          if (nc > 0) {
+            mma_commit(&B->c_empty[0]);
+            mma_commit(&B->c_empty[1]);
+          }
+          if (!km_wait(B, &B->c_full[nc % Cfg::CST], (nc / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA) ||
+              !km_wait(B, &B->c_full[(nc + 1) % Cfg::CST], ((nc + 1) / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t cb = smem_u32(smem + Cfg::OFF_C + cs * 2 * Cfg::C_BYTES);
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * Cfg::HALF + (kk & 3) * 32;
-              mma_bf16_ss(tmem + ab * Cfg::NC, smem_desc_sw128(xb + koff, 16, 1024),
-                          smem_desc_sw128(cb + part * Cfg::C_BYTES + koff, 16, 1024), Cfg::IDESC,
-                          (part == 0 && kk == 0) ? 0u : 1u);
+          nc += 2;
+          cur_h = h;
+        }
+        for (int j = 0; j < nchunks && ok; ++j) {
+          uint32_t c_hi = nc - 2, c_lo = nc - 1;   // SINGLE: the resident parts
+          if (!SINGLE) {
+            c_hi = nc;
+            c_lo = nc + 1;
+            if (!km_wait(B, &B->c_full[c_hi % Cfg::CST], (c_hi / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA) ||
+                !km_wait(B, &B->c_full[c_lo % Cfg::CST], (c_lo / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA)) {
+              ok = false;
+              break;
             }
           }
-          mma_commit(&B->c_empty[cs]);
-          mma_commit(&B->acc_full[ab]);
+          for (int t = 0; t < nt; ++t) {
+            const uint32_t xn = nx + t;
+            const int ab = 2 * t + static_cast<int>(kacc[t] & 1);
+            if ((j == 0 && !km_wait(B, &B->x_full[xn % Cfg::XST], (xn / Cfg::XST) & 1, wait_ns,
+                                    SITE_KMEANS_MMA)) ||
+                (kacc[t] >= 2 && !km_wait(B, &B->acc_empty[ab], ((kacc[t] >> 1) - 1) & 1, wait_ns,
+                                          SITE_KMEANS_MMA))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const SmemDesc xd{xd0.lo + (((xn % Cfg::XST) * Cfg::X_BYTES) >> 4), xd0.hi};
+            const SmemDesc hd{cd0.lo + (((c_hi % Cfg::CST) * Cfg::C_BYTES) >> 4), cd0.hi};
+            const SmemDesc ld{cd0.lo + (((c_lo % Cfg::CST) * Cfg::C_BYTES) >> 4), cd0.hi};
+            mma_chain<D / 16, Cfg::HALF, 32, Cfg::HALF, 32>(tmem + ab * Cfg::NC, xd, hd, Cfg::IDESC, 0u);
+            mma_chain<D / 16, Cfg::HALF, 32, Cfg::HALF, 32>(tmem + ab * Cfg::NC, xd, ld, Cfg::IDESC, 1u);
+            mma_commit(&B->acc_full[ab]);
+            ++kacc[t];
+            if (j == nchunks - 1) mma_commit(&B->x_empty[xn % Cfg::XST]);   // last reader of this x tile
+          }
+          if (!SINGLE && ok) {
+            mma_commit(&B->c_empty[c_hi % Cfg::CST]);
+            mma_commit(&B->c_empty[c_lo % Cfg::CST]);
+            nc += 2;
+          }
         }
-        if (ok) mma_commit(&B->x_empty[xs]);   // the unit's MMAs are the last readers of x
+        nx += nt;
+        u += nt;
       }
       mma_commit(&B->drain);
       mbar_wait(&B->drain, 0, 1000000000ull);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Two groups of four warps; group g takes the chunks with (global chunk
-    // index & 1) == g, from accumulator buffers g and g + 2 in turn.  Thread
-    // `row` of a group = token n0 + row = TMEM lane row.
+    // Group g owns tile g of every pair; thread `row` = token n0 + row = TMEM
+    // lane row.  Accumulators 2g and 2g + 1 alternate.
     //
     // Best two centroids per row with three min/max operations per score.
     // Every score s becomes a key: s with its low byte replaced by the
@@ -247,8 +299,7 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
     //   m2 = min(m2, max(m1, k)),  m1 = min(m1, k)
     // in two interleaved chains, and are then merged into the running best
     // and runner-up with the half-chunk's first column (an equal key keeps the
-    // earlier column).  When a unit has several chunks, group 1 hands its pair
-    // to group 0 through shared memory and group 0 merges.
+    // earlier column, chunks are taken in ascending order).
     // Near-tie rule: a key is within 2^-15 |s| of its score, and the
     // tensor-core score is within about 2^-16 (||x||^2 + ||mu||^2) of the
     // exact one (bf16 split residual and fp32 accumulation).  A runner-up
@@ -265,20 +316,21 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
 #pragma unroll
     for (int r = 0; r < 16; ++r)
       asm volatile("mov.b32 %0, %1;" : "=r"(colb[r]) : "r"(0x03020100u + 0x04040404u * r));
-    uint32_t nu = 0, gc = 0;
-    for (int u = blockIdx.x; u < units; u += grid, ++nu) {
+    uint32_t k = 0;   // accumulators this group has read
+    bool ok = true;
+    for (int u0 = u_begin; u0 < u_end && ok; ) {
+      const int nt = km_pair_tiles(u0, u_end, tiles);
+      const int u = u0 + grp;
+      u0 += nt;
+      if (grp >= nt) continue;
       const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
       const bool valid = n0 + row < N;
+      const float *nh = norms + static_cast<size_t>(h) * Cpad;
       float best = kBig, second = kBig;
       int arg = 0x7fffffff, arg2 = -1;
-      bool ok = true, mine_any = false;
-      for (int j = 0; j < nchunks; ++j, ++gc) {
-        if (static_cast<int>(gc & 1) != grp) continue;
-        const int ab = gc & 3;     // accumulator buffer and norms slot
-        mine_any = true;
-        const bool got = mbar_wait(&B->acc_full[ab], (gc >> 2) & 1, wait_ns) &&
-                         mbar_wait(&B->n_full[ab], (gc >> 2) & 1, wait_ns);
-        if (!__all_sync(0xffffffffu, got)) {
+      for (int j = 0; j < nchunks; ++j, ++k) {
+        const int ab = 2 * grp + static_cast<int>(k & 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(&B->acc_full[ab], (k >> 1) & 1, wait_ns))) {
           if (lane == 0) {
             record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
             atomicExch(&B->abort_flag, 1);
@@ -287,7 +339,7 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const float4 *nv4 = reinterpret_cast<const float4 *>(sNorm + ab * Cfg::NC);
+        const float4 *nv4 = reinterpret_cast<const float4 *>(nh + j * Cfg::NC);
         const uint32_t acc_addr = tmem + lane_off + ab * Cfg::NC;
         // 32-column pieces: the next piece's TMEM load is in flight while the
         // current one is reduced
@@ -307,19 +359,19 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
           const uint32_t *acc = buf[pc & 1];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 nv = nv4[pc * 8 + c4];
+            const float4 nv = __ldg(nv4 + pc * 8 + c4);
             const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float sc = fmaf(-2.f, __uint_as_float(acc[4 * c4 + e]), nn[e]);
-              const float k = __int_as_float(
+              const float kk = __int_as_float(
                   __byte_perm(__float_as_int(sc), colb[(pc & 1) * 8 + c4], 0x3214 + e));
               if (e & 1) {
-                q2 = fminf(q2, fmaxf(q1, k));
-                q1 = fminf(q1, k);
+                q2 = fminf(q2, fmaxf(q1, kk));
+                q1 = fminf(q1, kk);
               } else {
-                p2 = fminf(p2, fmaxf(p1, k));
-                p1 = fminf(p1, k);
+                p2 = fminf(p2, fmaxf(p1, kk));
+                p1 = fminf(p1, kk);
               }
             }
           }
@@ -340,60 +392,8 @@ __global__ void __launch_bounds__(KmCfg<D>::THREADS, 1)
           }
           if (pc < 3) tmem_wait32(buf[(pc + 1) & 1]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B->n_empty[ab]);
       }
       if (!__all_sync(0xffffffffu, ok)) break;
-      // combine the two groups' pairs when both saw chunks of this unit
-      bool owner = mine_any;
-      if (nchunks >= 2) {
-        const int ms = nu & 1;
-        float4 *slot = sMerge + ms * 128 + row;
-        if (grp == 1) {
-          if (nu >= 2 && !__all_sync(0xffffffffu, mbar_wait(&B->merge_empty[ms], ((nu >> 1) - 1) & 1, wait_ns))) {
-            if (lane == 0) {
-              record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
-              atomicExch(&B->abort_flag, 1);
-            }
-            break;
-          }
-          *slot = make_float4(best, __int_as_float(arg), second, __int_as_float(arg2));
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B->merge_full[ms]);
-          owner = false;
-        } else {
-          if (!__all_sync(0xffffffffu, mbar_wait(&B->merge_full[ms], (nu >> 1) & 1, wait_ns))) {
-            if (lane == 0) {
-              record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
-              atomicExch(&B->abort_flag, 1);
-            }
-            break;
-          }
-          const float4 o = *slot;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B->merge_empty[ms]);
-          const float ob = o.x, os = o.z;
-          const int oa = __float_as_int(o.y), oa2 = __float_as_int(o.w);
-          // top two (score, index) of the union of the two pairs
-          if (ob < best || (ob == best && oa < arg)) {
-            if (best < os || (best == os && arg < oa2)) {
-              second = best;
-              arg2 = arg;
-            } else {
-              second = os;
-              arg2 = oa2;
-            }
-            best = ob;
-            arg = oa;
-          } else if (ob < second || (ob == second && oa < arg2)) {
-            second = ob;
-            arg2 = oa;
-          }
-          owner = true;
-        }
-      }
-      if (!owner) continue;
-      const float *nh = norms + static_cast<size_t>(h) * Cpad;
       const bool live = valid && arg >= 0 && arg < C;
       if (valid && !live) record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);
       bool tie = false;

@@ -102,7 +102,7 @@ struct Carve {
   }
 };
 
-inline int kmeans_cpad(int C) { return (C + KmCfg<128>::NC - 1) / KmCfg<128>::NC * KmCfg<128>::NC; }
+inline int kmeans_cpad(int C) { return (C + kKmChunk - 1) / kKmChunk * kKmChunk; }
 
 struct KmeansWs {
   double *partial;
@@ -213,9 +213,47 @@ cudaEvent_t *prof_slot(int kernel) {
   return g_prof.ev[kernel][g_prof.used[kernel]++];
 }
 
+// (query tile, key tile) pairs the attention kernel issued MMAs for while
+// profiling was on; one counter per device (module-scope device storage).
+__device__ unsigned long long g_attn_issued_pairs = 0;
+
+constexpr int kMaxDevices = 64;
+void *g_issued_ptr[kMaxDevices] = {};
+
+// Device address of g_attn_issued_pairs on the current device (nullptr on failure).
+void *issued_pairs_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_prof_mutex);
+  if (g_issued_ptr[dev] == nullptr) {
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_issued_pairs);
+    if (e != cudaSuccess) {
+      cuda_status(e, "cudaGetSymbolAddress(attention pair counter)");
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_issued_ptr[dev] = ptr;
+  }
+  return g_issued_ptr[dev];
+}
+
 }  // namespace
 
 extern "C" {
+
+svg_status svg_profile_attn_pairs(uint64_t *pairs) {
+  if (!pairs) return SVG_ERR_INVALID_ARG;
+  unsigned long long v = 0, zero = 0;
+  svg_status st = cuda_status(cudaMemcpyFromSymbol(&v, g_attn_issued_pairs, sizeof(v)),
+                              "cudaMemcpyFromSymbol(attention pair counter)");
+  if (st != SVG_OK) return st;
+  st = cuda_status(cudaMemcpyToSymbol(g_attn_issued_pairs, &zero, sizeof(zero)),
+                   "cudaMemcpyToSymbol(attention pair counter)");
+  if (st != SVG_OK) return st;
+  *pairs = v;
+  return SVG_OK;
+}
 
 svg_status svg_profile_enable(int on) {
   std::lock_guard<std::mutex> lock(g_prof_mutex);
@@ -327,23 +365,30 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   const dim3 gb((N + 1024 * kBucketTokens - 1) / (1024 * kBucketTokens), BH);
   const dim3 gacc((max_accum_chunks(N, C) + 7) / 8, BH);
   int32_t *sizes = w.sizes(BH, C), *cursor = w.cursor(BH, C), *arrive = w.arrive(BH, C);
-  if (D == 128) {
-    if (!set_smem(kmeans_assign_tc_kernel<128>, KmCfg<128>::SMEM_BYTES)) return SVG_ERR_CUDA;
-  } else {
-    if (!set_smem(kmeans_assign_tc_kernel<64>, KmCfg<64>::SMEM_BYTES)) return SVG_ERR_CUDA;
-  }
+  // one centroid chunk (C <= 128): the chunk stays resident per head; more:
+  // tiles in pairs sharing every chunk
+  const bool single = Cpad == kKmChunk;
+  auto assign_kernel = [&](auto kernel, size_t smem_bytes, int threads) {
+    if (!set_smem(kernel, smem_bytes)) return SVG_ERR_CUDA;
+    kernel<<<ga, threads, smem_bytes, s>>>(mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign,
+                                          sizes, w.ties, w.num_ties, g_wait_ns);
+    return launch_status("kmeans_assign_tc_kernel");
+  };
   for (int it = 0; it < iters; ++it) {
     cudaEvent_t *pe = prof_slot(0);
     if (pe) cudaEventRecord(pe[0], s);
+    svg_status st;
     if (D == 128)
-      kmeans_assign_tc_kernel<128><<<ga, KmCfg<128>::THREADS, KmCfg<128>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, sizes, w.ties, w.num_ties,
-          g_wait_ns);
+      st = single ? assign_kernel(kmeans_assign_tc_kernel<128, true>, KmCfg<128, true>::SMEM_BYTES,
+                                  KmCfg<128, true>::THREADS)
+                  : assign_kernel(kmeans_assign_tc_kernel<128, false>, KmCfg<128, false>::SMEM_BYTES,
+                                  KmCfg<128, false>::THREADS);
     else
-      kmeans_assign_tc_kernel<64><<<ga, KmCfg<64>::THREADS, KmCfg<64>::SMEM_BYTES, s>>>(
-          mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign, sizes, w.ties, w.num_ties,
-          g_wait_ns);
-    if (launch_status("kmeans_assign_tc_kernel") != SVG_OK) return SVG_ERR_CUDA;
+      st = single ? assign_kernel(kmeans_assign_tc_kernel<64, true>, KmCfg<64, true>::SMEM_BYTES,
+                                  KmCfg<64, true>::THREADS)
+                  : assign_kernel(kmeans_assign_tc_kernel<64, false>, KmCfg<64, false>::SMEM_BYTES,
+                                  KmCfg<64, false>::THREADS);
+    if (st != SVG_OK) return st;
     if (pe) cudaEventRecord(pe[1], s);
     if (D == 128)
       kmeans_refine_kernel<128><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
@@ -416,20 +461,32 @@ svg_status svg_select_topp(const float *mu_q, const int32_t *n_q, const float *m
   if (BH <= 0 || Cq <= 0 || Ck <= 0 || !(p > 0.f) || std::isnan(p)) return SVG_ERR_INVALID_ARG;
   if (Ck > kMaxCk || (D != 64 && D != 128)) return SVG_ERR_UNSUPPORTED;
   if (!aligned(mu_q, 16) || !aligned(mu_k, 16)) return SVG_ERR_INVALID_ARG;
-  if (!(scale > 0.f)) scale = 1.f / std::sqrt(static_cast<float>(D));
+  // the default scale is formed in float64 (1/sqrt(D) correctly rounded), the
+  // precision the cut is decided in
+  const double scale_d = scale > 0.f ? static_cast<double>(scale) : 1.0 / std::sqrt(static_cast<double>(D));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t smem = select_smem_bytes(D, Ck);
-  const dim3 grid((Cq + kRowsPerBlock - 1) / kRowsPerBlock, BH);
+  const dim3 grid((Cq + kSelRows - 1) / kSelRows, BH);
+  const int cpl = select_cpl(Ck);
+  auto launch = [&](auto kernel) {
+    if (!set_smem(kernel, smem)) return SVG_ERR_CUDA;
+    kernel<<<grid, kSelRows * 32, smem, s>>>(mu_q, n_q, mu_k, n_k, Cq, Ck, p, scale_d, sel_count, sel_cols);
+    return launch_status("select_topp_kernel");
+  };
   if (D == 128) {
-    if (!set_smem(select_topp_kernel<128>, smem)) return SVG_ERR_CUDA;
-    select_topp_kernel<128><<<grid, 256, smem, s>>>(mu_q, n_q, mu_k, n_k, Cq, Ck, p, scale,
-                                                    sel_count, sel_cols);
-  } else {
-    if (!set_smem(select_topp_kernel<64>, smem)) return SVG_ERR_CUDA;
-    select_topp_kernel<64><<<grid, 256, smem, s>>>(mu_q, n_q, mu_k, n_k, Cq, Ck, p, scale,
-                                                   sel_count, sel_cols);
+    switch (cpl) {
+      case 4: return launch(select_topp_kernel<128, 4>);
+      case 8: return launch(select_topp_kernel<128, 8>);
+      case 16: return launch(select_topp_kernel<128, 16>);
+      default: return launch(select_topp_kernel<128, 32>);
+    }
   }
-  return launch_status();
+  switch (cpl) {
+    case 4: return launch(select_topp_kernel<64, 4>);
+    case 8: return launch(select_topp_kernel<64, 8>);
+    case 16: return launch(select_topp_kernel<64, 16>);
+    default: return launch(select_topp_kernel<64, 32>);
+  }
 }
 
 // ------------------------------------------------------------------ sparse attention
@@ -455,6 +512,7 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   if (perm != nullptr && (op == qp || op == kp || op == vp)) return SVG_ERR_INVALID_ARG;
   if (!sizes_ok(BH, N) || Cq < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (Ck > AttnCfg<128>::MAX_SEL) return SVG_ERR_UNSUPPORTED;
   if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16) ||
       !aligned(ws, 256))
     return SVG_ERR_INVALID_ARG;
@@ -465,8 +523,9 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
   const int pairs = BH * Cq;
+  const int max_sel = Ck < AttnCfg<128>::MAX_SEL ? Ck : AttnCfg<128>::MAX_SEL;
   attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
-                                                            Cq, Ck, w.qtiles, w.ktiles);
+                                                            Cq, Ck, max_sel, w.qtiles, w.ktiles);
   attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, w.items,
                                                    w.num_items, w.next_item);
   svg_status st = launch_status();
@@ -490,6 +549,11 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   prm.op = static_cast<__nv_bfloat16 *>(op);
   prm.lse = lse;
   prm.perm = perm;
+  prm.issued = nullptr;
+  if (g_prof.on) {
+    prm.issued = static_cast<unsigned long long *>(issued_pairs_address());
+    if (prm.issued == nullptr) return SVG_ERR_CUDA;
+  }
   prm.N = N;
   prm.Cq = Cq;
   prm.Ck = Ck;
@@ -546,7 +610,6 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
 namespace {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SVG_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 void *g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mutex;
 
@@ -557,7 +620,12 @@ void *noalloc_scratch_address() {
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (g_noalloc_ptr[dev] == nullptr) {
     void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      cuda_status(e, "cudaGetSymbolAddress(no-allocation scratch)");   // recorded for svg_last_cuda_error
+      cudaGetLastError();                                              // and not left pending
+      return nullptr;
+    }
     g_noalloc_ptr[dev] = ptr;
   }
   return g_noalloc_ptr[dev];

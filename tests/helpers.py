@@ -12,6 +12,11 @@ ATTN_MAX_ABS = 2e-2
 KMEANS_AGREE = 0.999
 
 
+def as_f32(p: float) -> float:
+    """The float32 value a float argument of the C ABI carries (e.g. top-p)."""
+    return float(np.float32(p))
+
+
 def dev_bf16(x: np.ndarray) -> torch.Tensor:
     """bfloat16-valued float32 array -> bit-identical CUDA bf16 tensor."""
     bits = synth.bf16_bits(x).view(np.int16)

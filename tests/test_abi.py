@@ -83,8 +83,9 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
     assert lib.svg_select_topp(f, f, f, f, 1, 4, 8, 64, 0.0, 0.0, f, f, nul) == 1
     assert lib.svg_select_topp(f, f, f, f, 1, 4, 8, 64, float("nan"), 0.0, f, f, nul) == 1
     assert lib.svg_select_topp(f, f, f, f, 1, 4, 2048, 64, 0.9, 0.0, f, f, nul) == 2
-    # attention: unsupported D, workspace too small
+    # attention: unsupported D, more than 1024 k-clusters, workspace too small
     assert lib.svg_sparse_attn(f, f, f, 1, 16, 80, f, 2, f, 2, f, f, 0.0, f, nul, f, 1 << 20, nul) == 2
+    assert lib.svg_sparse_attn(f, f, f, 1, 4096, 64, f, 2, f, 1025, f, f, 0.0, f, nul, f, 1 << 20, nul) == 2
     assert lib.svg_sparse_attn(f, f, f, 1, 4096, 64, f, 2, f, 2, f, f, 0.0, f, nul, f, 8, nul) == 3
     # fused attention + un-permute: missing perm_q, output aliasing an input, small workspace
     g = _p(FAKE + 4096)

@@ -68,3 +68,19 @@ def test_device_check_reports_bad_block_list():
     svg.sparse_attn(st.qp, st.kp, st.vp, st.q_off, st.k_off, st.sel_count, cols)
     assert svg.get_error() == 6                      # SVG_ERR_DEVICE_CHECK
     assert svg.get_error() == 0
+
+
+def test_device_check_reports_block_count_beyond_the_row():
+    """A block count above Ck is clamped to the row (no read past it) and flagged."""
+    wl = synth.small_workload("480p-5s", (5, 12, 20), heads=1, cq=6, ck=40, iters=2)
+    L = synth.make_layer(wl)
+    layer = svg.SvgLayer(*L.q.shape, wl.cq, wl.ck)
+    _, st = layer(dev_bf16(L.q), dev_bf16(L.k), dev_bf16(L.v), dev_f32(L.init_centroids("q")),
+                  dev_f32(L.init_centroids("k")), wl.iters, 0.9)
+    cnt = st.sel_count.clone()
+    cols = torch.arange(wl.ck, dtype=torch.int32, device=cnt.device).expand_as(st.sel_cols).contiguous()
+    i = int(np.nonzero(cnt.cpu().numpy()[0] > 0)[0][-1])   # the last non-empty row: nothing follows it
+    cnt[0, i] = wl.ck + 1
+    svg.sparse_attn(st.qp, st.kp, st.vp, st.q_off, st.k_off, cnt, cols)
+    assert svg.get_error() == 6                      # SVG_ERR_DEVICE_CHECK
+    assert svg.get_error() == 0
