@@ -21,28 +21,38 @@
 // accumulators instruction by instruction costs ~150 cycles per MMA; so the
 // kernel issues whole chains and never interleaves them.
 //
-// Per CTA (persistent, one per SM), 11 warps:
+// Per CTA (persistent, one per SM), 12 warps:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t owns
 //              query row t of its tile (TMEM lane t)
-//   warp 8     TMA producer: Q tiles; K and V tiles through one ring, in the
-//              order the MMAs consume them: K0, K1, V0, K2, V1, ..., V(n-1)
-//   warp 9     MMA issuer: walks the same sequence; for a K entry issues
-//              S_x = Q_x K^T of both tiles, for a V entry O_x += P_x V; owns TMEM
+//   warp 8     TMA producer: Q tiles; K and V tiles of every key tile into
+//              two rings (two slots each at D = 128)
+//   warps 9, 11 MMA issuers, one per query tile (warp 9 owns TMEM): the
+//              sequence S(0), PV(0), S(1), PV(1), ... with S_x = Q_x K^T (A and
+//              B in shared memory) and O_x += P_x V (A = P in tensor memory)
 //   warp 10    item loader: claims the next item from a counter shared by all
 //              CTAs (list sorted by head group, then longest first), prefetches
 //              its query rows into L2, merges its key ranges into runs
-// S_x has one TMEM buffer per tile; the softmax copies it to registers and
-// releases it at once, so S_x(t+1) runs on the tensor cores while the softmax
-// of tile t computes.  P is written by the softmax warps to shared memory
-// (bf16, 128-byte swizzled, K-major), so both MMAs read shared memory.  O
-// accumulates in TMEM across the item's key tiles; the softmax warps rescale
-// it in place only when a row's running max grows by more than 2^8 (exact:
-// every probability is taken against the same reference max that O and the
-// row sum use).
+// Tensor memory per query tile x: S_x (128 fp32 columns) and O_x (D
+// columns).  The softmax reads S_x(t) into registers and writes P_x(t) as
+// bf16 pairs over the first 64 columns of S_x, where the PV MMA takes it as
+// its A operand; S_x(t+1) is issued after PV_x(t), and MMAs run in issue
+// order, so it overwrites P only after PV has read it.  The two query tiles
+// alternate on the tensor pipe: one tile's MMAs run while the other's
+// softmax computes.  O accumulates in TMEM across the item's key tiles; the
+// softmax warps rescale it in place only when a row's running max grows by
+// more than 2^8 (exact: every probability is taken against the same
+// reference max that O and the row sum use).
 #pragma once
 #include "common.cuh"
 
 namespace svg {
+
+#ifndef SVG_EXP_POLY_PAIRS
+#define SVG_EXP_POLY_PAIRS 0
+#endif
+#ifndef SVG_PACK_INT
+#define SVG_PACK_INT 0
+#endif
 
 constexpr int kItemRows = 256;     // query rows per work item (two 128-row tiles)
 constexpr int kSlotsPerTile = 16;  // 8-row slots per 128-key tile
@@ -53,33 +63,32 @@ struct AttnItem {  // up to 256 query rows of one q-cluster; h < 0 ends the list
 };
 
 // Readers of an item header slot that must release it before it is refilled:
-// the producer, the MMA issuer and the eight softmax warps.
-constexpr int kItemReaders = 10;
+// the producer, the two MMA issuers and the eight softmax warps.
+constexpr int kItemReaders = 11;
 
 template <int D>
 struct AttnCfg {
   static constexpr int BM = 128, BN = 128, SLOT = 8, NSLOT = BN / SLOT;
   static constexpr int DH = D / 64;                   // 64-channel (128-byte) halves
-  static constexpr int KVST = D == 128 ? 2 : 4;       // K/V ring slots
+  static constexpr int KST = D == 128 ? 2 : 4;        // K ring slots (same for V)
   static constexpr int QT_BYTES = BM * D * 2;         // one Q tile
   static constexpr int KV_BYTES = BN * D * 2;         // one K or V tile
-  static constexpr int P_BYTES = BM * BN * 2;         // one P tile
   static constexpr int HALF_Q = BM * 128;             // one 64-channel half of a Q tile
   static constexpr int HALF_KV = BN * 128;            // same for a K/V tile
-  static constexpr int HALF_P = BM * 128;             // one 64-key half of a P tile
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + 2 * QT_BYTES;
-  static constexpr int OFF_P = OFF_KV + KVST * KV_BYTES;
+  static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int MAX_SEL = 1024;                // selected k-clusters per q-cluster
-  static constexpr int OFF_RANGES = OFF_P + 2 * P_BYTES;   // int2 (first row, rows) per run
+  static constexpr int OFF_RANGES = OFF_V + KST * KV_BYTES;   // int2 (first row, rows) per run
   static constexpr int OFF_BAR = OFF_RANGES + MAX_SEL * 8;
   static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers/meta + alignment slack
-  // TMEM: S of tile x at x*128 (128 columns); O of tile x at 256 + x*128
+  // TMEM: S (then P) of tile x at x*128 (128 columns); O of tile x at 256 + x*128
   static constexpr uint32_t TM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, LOADER_WARP = 10;
-  static constexpr int THREADS = 11 * 32;
+  // warp 9 issues tile A's MMAs (and owns TMEM), warp 11 tile B's
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, LOADER_WARP = 10, MMA_B_WARP = 11;
+  static constexpr int THREADS = 12 * 32;
   __device__ static constexpr uint32_t tm_s(int x) { return x * 128; }
   __device__ static constexpr uint32_t tm_o(int x) { return 256 + x * 128; }
 };
@@ -117,13 +126,15 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count)
 }
 
 struct AttnBarriers {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[4], kv_empty[4];
+  uint64_t q_full, q_empty[2];                      // q_empty: [tile]
+  uint64_t k_full[4], v_full[4];
+  uint64_t k_empty[2][4], v_empty[2][4];            // [tile][slot]: released by that tile's MMAs
   uint64_t meta_full[kMetaRing];
-  uint64_t s_full[2], s_free[2], p_full[2], o_full[2];   // [tile]
+  uint64_t s_full[2], p_full[2], o_full[2];   // [tile]
+  uint64_t exp_done[2];                       // [tile]: its four softmax warps finished a step's exponentials
   uint64_t item_full[2], item_empty[2];
   uint64_t ranges_full, ranges_empty;
-  uint64_t drain;
+  uint64_t drain[2];
   AttnItem item[2];      // item header ring written by the loader warp
   int32_t ranges_cnt;    // runs of the item whose ranges are in shared memory
   uint32_t meta[kMetaRing][4];   // per key tile: 128-bit key validity mask
@@ -194,8 +205,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = smem + Cfg::OFF_Q;
-  uint8_t *sKV = smem + Cfg::OFF_KV;
-  uint8_t *sP = smem + Cfg::OFF_P;
+  uint8_t *sK = smem + Cfg::OFF_K;
+  uint8_t *sV = smem + Cfg::OFF_V;
   int2 *sRanges = reinterpret_cast<int2 *>(smem + Cfg::OFF_RANGES);
   AttnBarriers *B = reinterpret_cast<AttnBarriers *>(smem + Cfg::OFF_BAR);
   const int warp = static_cast<int>(warp_id());
@@ -203,23 +214,27 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&B->q_full, 1);
-    mbar_init(&B->q_empty, 1);
     for (int s = 0; s < 4; ++s) {
-      mbar_init(&B->kv_full[s], 1);
-      mbar_init(&B->kv_empty[s], 1);
+      mbar_init(&B->k_full[s], 1);
+      mbar_init(&B->v_full[s], 1);
+      for (int x = 0; x < 2; ++x) {
+        mbar_init(&B->k_empty[x][s], 1);
+        mbar_init(&B->v_empty[x][s], 1);
+      }
     }
     for (int s = 0; s < kMetaRing; ++s) mbar_init(&B->meta_full[s], 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&B->s_full[x], 1);
-      mbar_init(&B->s_free[x], 4);
       mbar_init(&B->p_full[x], 4);
+      mbar_init(&B->exp_done[x], 4);
       mbar_init(&B->o_full[x], 1);
       mbar_init(&B->item_full[x], 1);
       mbar_init(&B->item_empty[x], kItemReaders);
+      mbar_init(&B->q_empty[x], 1);
+      mbar_init(&B->drain[x], 1);
     }
     mbar_init(&B->ranges_full, 1);
     mbar_init(&B->ranges_empty, 1);
-    mbar_init(&B->drain, 1);
     B->abort_flag = 0;
     fence_mbar_init();
   }
@@ -307,9 +322,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
   } else if (warp == Cfg::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
+    // Per item: the Q tiles, then K(t) and V(t) of every key tile t (both
+    // through the same box list).  K(t + KST) waits for S(t) of both query
+    // tiles, V(t + KST) for PV(t).
     uint32_t g = 0;         // global key-tile counter
-    uint32_t e = 0;         // global ring-entry counter (K and V tiles issued)
     uint32_t nq = 0;        // Q loads issued (for the drain)
+    uint32_t gk = 0, gv = 0;   // K and V tiles issued (for the drain)
+    // A slot (and Q) is reused once every query tile of its last occupant has
+    // released it: tile A is in every item, tile B only in items of > 128
+    // rows; slot_b[s] = whether the slot's last occupant had tile B,
+    // rel_b[s] / nq_b = tile-B releases of the slot / of Q expected so far.
+    bool slot_b[4] = {false, false, false, false}, prev_b = false;
+    uint32_t rel_b[4] = {0, 0, 0, 0}, nq_b = 0;
     if (lane == 0) {
       bool ok = true;
       for (int n = 0; ok && !aborted(B); ++n) {
@@ -324,7 +348,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const int cnt = B->ranges_cnt;
         const int ntk = it.packed >> 9;
         const bool has_b = (it.packed & 0x1FF) > Cfg::BM;
-        if (n > 0 && !attn_wait(B, &B->q_empty, (n - 1) & 1, ns, SITE_ATTN_PRODUCER)) break;
+        if (n > 0 && (!attn_wait(B, &B->q_empty[0], (n - 1) & 1, ns, SITE_ATTN_PRODUCER) ||
+                      (prev_b && !attn_wait(B, &B->q_empty[1], (nq_b - 1) & 1, ns, SITE_ATTN_PRODUCER))))
+          break;
+        prev_b = has_b;
+        if (has_b) ++nq_b;
         if (P.fault != 1) {
           mbar_arrive_expect_tx(&B->q_full, Cfg::QT_BYTES * (has_b ? 2 : 1));
           const int qrow = it.h * P.N + it.q0;
@@ -338,68 +366,72 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
           ++nq;
         }
-        // box lists of the last two key tiles (a V tile is issued after the
-        // next tile's K): row and (kind | slot << 8) of every box
-        int box_row[2][Cfg::NSLOT], box_kind[2][Cfg::NSLOT], nbox[2] = {0, 0};
         int ci = 0, cur = 0, left = 0;
         const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
-        for (int en = 0; en < 2 * ntk && ok; ++en) {
-          bool is_k;
-          const int t = attn_entry(ntk, en, is_k);
-          const int lb = t & 1;
-          if (is_k) {
-            // cut tile t into boxes of 1..16 slots (8..128 rows): the largest
-            // power of two that fits both the tile and the rest of the run
-            uint32_t mask[4] = {0, 0, 0, 0};
-            int sl = 0, nb = 0;
-            while (sl < Cfg::NSLOT) {
-              while (left <= 0 && ci < cnt) {
-                const int2 r = sRanges[ci++];
-                cur = r.x;
-                left = r.y;
-              }
-              const int space = Cfg::NSLOT - sl;
-              const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
-              int kind = 0;
-              while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
-              const int nsl = 1 << kind;
-              if (left > 0) {
-                set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
-                box_row[lb][nb] = it.h * P.N + cur;
-                cur += nsl * Cfg::SLOT;
-                left -= nsl * Cfg::SLOT;
-              } else {
-                box_row[lb][nb] = pad_row;   // no keys left: finite filler rows, masked out
-              }
-              box_kind[lb][nb] = kind | (sl << 8);
-              ++nb;
-              sl += nsl;
+        for (int t = 0; t < ntk && ok; ++t, ++g) {
+          // cut tile t into boxes of 1..16 slots (8..128 rows): the largest
+          // power of two that fits both the tile and the rest of the run
+          int box_row[Cfg::NSLOT], box_kind[Cfg::NSLOT], nb = 0;
+          uint32_t mask[4] = {0, 0, 0, 0};
+          int sl = 0;
+          while (sl < Cfg::NSLOT) {
+            while (left <= 0 && ci < cnt) {
+              const int2 r = sRanges[ci++];
+              cur = r.x;
+              left = r.y;
             }
-            nbox[lb] = nb;
-            if (t == ntk - 1) mbar_arrive(&B->ranges_empty);   // the ranges are no longer read
-            const int mi = static_cast<int>(g % kMetaRing);
+            const int space = Cfg::NSLOT - sl;
+            const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
+            int kind = 0;
+            while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
+            const int nsl = 1 << kind;
+            if (left > 0) {
+              set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
+              box_row[nb] = it.h * P.N + cur;
+              cur += nsl * Cfg::SLOT;
+              left -= nsl * Cfg::SLOT;
+            } else {
+              box_row[nb] = pad_row;   // no keys left: finite filler rows, masked out
+            }
+            box_kind[nb] = kind | (sl << 8);
+            ++nb;
+            sl += nsl;
+          }
+          if (t == ntk - 1) mbar_arrive(&B->ranges_empty);   // the ranges are no longer read
+          const int mi = static_cast<int>(g % kMetaRing);
 #pragma unroll
-            for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
-            mbar_arrive(&B->meta_full[mi]);
-            ++g;
-          }
-          const int slot = static_cast<int>(e % Cfg::KVST);
-          if (e >= static_cast<uint32_t>(Cfg::KVST) &&
-              !attn_wait(B, &B->kv_empty[slot], ((e / Cfg::KVST) - 1) & 1, ns, SITE_ATTN_PRODUCER)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&B->kv_full[slot], Cfg::KV_BYTES);
-          uint8_t *dst = sKV + slot * Cfg::KV_BYTES;
-          const CUtensorMap *maps_t = is_k ? maps.k : maps.v;
-          for (int bx = 0; bx < nbox[lb]; ++bx) {
-            const int kind = box_kind[lb][bx] & 0xFF, at = box_kind[lb][bx] >> 8;
+          for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
+          mbar_arrive(&B->meta_full[mi]);
+          const int slot = static_cast<int>(g % Cfg::KST);
+          const uint32_t ph = ((g / Cfg::KST) - 1) & 1;
+          const bool reuse_b = g >= static_cast<uint32_t>(Cfg::KST) && slot_b[slot];
+          const uint32_t ph_b = (rel_b[slot] - 1) & 1;
 #pragma unroll
-            for (int dh = 0; dh < Cfg::DH; ++dh)
-              tma_load_2d(dst + dh * Cfg::HALF_KV + at * 1024, &maps_t[kind], dh * 64, box_row[lb][bx],
-                          &B->kv_full[slot]);
+          for (int kv = 0; kv < 2; ++kv) {     // K(t), then V(t)
+            uint64_t *full = kv ? &B->v_full[slot] : &B->k_full[slot];
+            if (g >= static_cast<uint32_t>(Cfg::KST) &&
+                (!attn_wait(B, kv ? &B->v_empty[0][slot] : &B->k_empty[0][slot], ph, ns, SITE_ATTN_PRODUCER) ||
+                 (reuse_b && !attn_wait(B, kv ? &B->v_empty[1][slot] : &B->k_empty[1][slot], ph_b, ns,
+                                        SITE_ATTN_PRODUCER)))) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full, Cfg::KV_BYTES);
+            uint8_t *dst = (kv ? sV : sK) + slot * Cfg::KV_BYTES;
+            const CUtensorMap *maps_t = kv ? maps.v : maps.k;
+            for (int bx = 0; bx < nb; ++bx) {
+              const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
+#pragma unroll
+              for (int dh = 0; dh < Cfg::DH; ++dh)
+                tma_load_2d(dst + dh * Cfg::HALF_KV + at * 1024, &maps_t[kind], dh * 64, box_row[bx], full);
+            }
+            if (kv)
+              gv = g + 1;
+            else
+              gk = g + 1;
           }
-          ++e;
+          slot_b[slot] = has_b;
+          if (has_b) ++rel_b[slot];
         }
         mbar_arrive(&B->item_empty[buf]);
       }
@@ -407,111 +439,74 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       // last phase of each so no copy is in flight when the CTA exits.
       if (aborted(B)) {
         if (nq > 0) mbar_wait(&B->q_full, (nq - 1) & 1, 1000000000ull);
-        for (uint32_t k = (e >= static_cast<uint32_t>(Cfg::KVST) ? e - Cfg::KVST : 0); k < e; ++k)
-          mbar_wait(&B->kv_full[k % Cfg::KVST], (k / Cfg::KVST) & 1, 1000000000ull);
+        for (uint32_t k = (gk >= static_cast<uint32_t>(Cfg::KST) ? gk - Cfg::KST : 0); k < gk; ++k)
+          mbar_wait(&B->k_full[k % Cfg::KST], (k / Cfg::KST) & 1, 1000000000ull);
+        for (uint32_t k = (gv >= static_cast<uint32_t>(Cfg::KST) ? gv - Cfg::KST : 0); k < gv; ++k)
+          mbar_wait(&B->v_full[k % Cfg::KST], (k / Cfg::KST) & 1, 1000000000ull);
       }
     }
-  } else if (warp == Cfg::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    // Walks the ring entries in the producer's order.  For a K entry it
-    // issues S_x = Q_x K^T for each present tile x once S_x's buffer has been
-    // read by the softmax; for a V entry O_x += P_x V once P_x is written.
-    // The two tiles of an entry are issued independently (whichever is ready
-    // first); the ring slot is released when both have been issued.
+  } else if (warp == Cfg::MMA_WARP || warp == Cfg::MMA_B_WARP) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread per query tile x issues that tile's sequence S(0), PV(0),
+    // S(1), PV(1), ... of every item that has the tile: S_x(t) once K(t) (and
+    // Q) has landed, PV_x(t) once the softmax has written P_x(t) and V(t) has
+    // landed.  It releases each K/V slot and Q for its own tile; the producer
+    // reuses them when every present tile has released them.  Two issuers let
+    // one tile's chain queue on the tensor pipe while the other's executes.
+    const int x = warp == Cfg::MMA_WARP ? 0 : 1;
     if (lane == 0) {
-      // descriptors built once: Q and P tiles (per query tile), ring slot 0 as a
-      // K operand (K-major) and as a V operand (MN-major); a slot adds its offset
-      const SmemDesc qd[2] = {make_desc_sw128(smem_u32(sQ), 16, 1024),
-                              make_desc_sw128(smem_u32(sQ) + Cfg::QT_BYTES, 16, 1024)};
-      const SmemDesc pd[2] = {make_desc_sw128(smem_u32(sP), 16, 1024),
-                              make_desc_sw128(smem_u32(sP) + Cfg::P_BYTES, 16, 1024)};
-      const SmemDesc kd0 = make_desc_sw128(smem_u32(sKV), 16, 1024);
-      const SmemDesc vd0 = make_desc_sw128(smem_u32(sKV), Cfg::HALF_KV, 1024);
-      uint32_t n_hdr = 0, n_item = 0, e = 0;
-      uint32_t n_s[2] = {0, 0}, n_pv[2] = {0, 0};
-      bool have = false, finished = false, q_ok = false;
-      bool done[2] = {false, false};
-      int ntk = 0, en = 0;
-      bool has_b = false;
+      const SmemDesc qd = make_desc_sw128(smem_u32(sQ) + x * Cfg::QT_BYTES, 16, 1024);
+      const SmemDesc kd0 = make_desc_sw128(smem_u32(sK), 16, 1024);
+      const SmemDesc vd0 = make_desc_sw128(smem_u32(sV), Cfg::HALF_KV, 1024);
+      uint32_t g0 = 0, n_pv = 0;   // key tiles of earlier items; PV chains issued
       unsigned long long pairs = 0;
-      const long long limit = static_cast<long long>(ns) * 2;
-      long long t_last = clock64();
-      while (!finished) {
-        bool progress = false;
-        if (!have && mbar_test(&B->item_full[n_hdr & 1], (n_hdr >> 1) & 1)) {
-          const AttnItem it = B->item[n_hdr & 1];
-          mbar_arrive(&B->item_empty[n_hdr & 1]);
-          ++n_hdr;
-          if (it.h < 0) {
-            finished = true;
+      for (uint32_t n = 0; !aborted(B); ++n) {
+        if (!attn_wait(B, &B->item_full[n & 1], (n >> 1) & 1, ns, SITE_ATTN_MMA)) break;
+        const AttnItem it = B->item[n & 1];
+        mbar_arrive(&B->item_empty[n & 1]);
+        if (it.h < 0) break;
+        const int ntk = it.packed >> 9;
+        if (x == 1 && (it.packed & 0x1FF) <= Cfg::BM) {   // no tile B in this item
+          g0 += ntk;
+          continue;
+        }
+        if (!attn_wait(B, &B->q_full, n & 1, ns, SITE_ATTN_MMA)) break;
+        bool ok = true;
+        for (int t = 0; t < ntk && ok; ++t) {
+          const uint32_t gt = g0 + t;
+          const int slot = static_cast<int>(gt % Cfg::KST);
+          const uint32_t ph = (gt / Cfg::KST) & 1;
+          const uint32_t slot_off = (slot * Cfg::KV_BYTES) >> 4;
+          if (!attn_wait(B, &B->k_full[slot], ph, ns, SITE_ATTN_MMA)) { ok = false; break; }
+          tc_fence_after();
+          mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
+              tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
+          mma_commit(&B->s_full[x]);
+          mma_commit(&B->k_empty[x][slot]);
+          if (t == ntk - 1) mma_commit(&B->q_empty[x]);   // the item's last S: Q may be replaced
+          if (!attn_wait(B, &B->p_full[x], n_pv & 1, ns, SITE_ATTN_MMA) ||
+              !attn_wait(B, &B->v_full[slot], ph, ns, SITE_ATTN_MMA)) {
+            ok = false;
             break;
           }
-          ntk = it.packed >> 9;
-          has_b = (it.packed & 0x1FF) > Cfg::BM;
-          en = 0;
-          q_ok = false;
-          have = true;
-          progress = true;
+          tc_fence_after();
+          // A = P_x [128 q x 128 keys] in TMEM (the first 64 columns of S_x);
+          // B = V [128 keys x D], MN-major, 16 keys = 2048 bytes per K-step
+          mma_chain_ts<Cfg::BN / 16, 4 * 2048, 2048>(tmem + Cfg::tm_o(x), tmem + Cfg::tm_s(x),
+                                                     SmemDesc{vd0.lo + slot_off, vd0.hi}, Cfg::IDESC_PV,
+                                                     t > 0 ? 1u : 0u);
+          if (t == ntk - 1) mma_commit(&B->o_full[x]);   // the item's O of tile x is final
+          mma_commit(&B->v_empty[x][slot]);
+          ++n_pv;
+          ++pairs;
         }
-        if (have) {
-          bool is_k;
-          const int t = attn_entry(ntk, en, is_k);
-          const int slot = static_cast<int>(e % Cfg::KVST);
-          if (mbar_test(&B->kv_full[slot], (e / Cfg::KVST) & 1)) {
-            const uint32_t slot_off = (slot * Cfg::KV_BYTES) >> 4;
-            if (is_k && !q_ok) q_ok = mbar_test(&B->q_full, n_item & 1);
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              if (done[x] || (x == 1 && !has_b)) continue;
-              if (is_k) {
-                if (!q_ok) continue;
-                if (n_s[x] >= 1 && !mbar_test(&B->s_free[x], (n_s[x] - 1) & 1)) continue;
-                tc_fence_after();
-                mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
-                    tmem + Cfg::tm_s(x), qd[x], SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
-                mma_commit(&B->s_full[x]);
-                ++n_s[x];
-              } else {
-                if (!mbar_test(&B->p_full[x], n_pv[x] & 1)) continue;
-                tc_fence_after();
-                // A = P_x [128 q x 128 keys], K-major in two 64-key halves; B = V [128 keys x D],
-                // MN-major, 16 keys = 2048 bytes per K-step
-                mma_chain<Cfg::BN / 16, Cfg::HALF_P, 32, 4 * 2048, 2048>(
-                    tmem + Cfg::tm_o(x), pd[x], SmemDesc{vd0.lo + slot_off, vd0.hi}, Cfg::IDESC_PV,
-                    t > 0 ? 1u : 0u);
-                mma_commit(&B->o_full[x]);
-                ++n_pv[x];
-                ++pairs;
-              }
-              done[x] = true;
-              progress = true;
-            }
-            if (done[0] && (done[1] || !has_b)) {
-              mma_commit(&B->kv_empty[slot]);
-              if (is_k && t == ntk - 1) mma_commit(&B->q_empty);   // the item's last S: Q may be replaced
-              ++e;
-              done[0] = done[1] = false;
-              if (++en == 2 * ntk) {
-                have = false;
-                ++n_item;
-              }
-            }
-          }
-        }
-        if (progress) {
-          t_last = clock64();
-        } else if (clock64() - t_last > limit) {
-          record_error(SVG_ERR_TIMEOUT, SITE_ATTN_MMA);
-          atomicExch(&B->abort_flag, 1);
-          break;
-        } else if (aborted(B)) {
-          break;
-        }
+        if (!ok) break;
+        g0 += ntk;
       }
       if (P.issued != nullptr && pairs > 0) atomicAdd(P.issued, pairs);
       // make sure every issued MMA has retired before TMEM is released
-      mma_commit(&B->drain);
-      mbar_wait(&B->drain, 0, 1000000000ull);
+      mma_commit(&B->drain[x]);
+      mbar_wait(&B->drain[x], 0, 1000000000ull);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax warps
@@ -525,9 +520,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t o_addr = tmem + lane_off + Cfg::tm_o(x);
-    uint8_t *sPx = sP + x * Cfg::P_BYTES;
+    const uint32_t s_addr = tmem + lane_off + Cfg::tm_s(x);
     const float sl2 = P.scale_log2;
     uint32_t g = 0, n_s = 0, n_o = 0;
+    // Exponentials take turns between the two tiles of an item (A(t), B(t),
+    // A(t+1), ...), so one tile's exponentials overlap the other tile's MMAs
+    // instead of competing for the same MUFU units.  exp_done[y] completes
+    // once per step of tile y; other_before counts the other tile's steps in
+    // earlier items (tile A runs every item, tile B only items of > 128 rows).
+    // Neither tile can get two completions ahead of the other's wait: tile B
+    // waits for A(t) before finishing B(t), A waits for B(t-1) before A(t),
+    // and an item's first S is issued only after both tiles' last PV.
+    uint32_t other_before = 0;
     for (uint32_t n = 0; !warp_aborted(B); ++n) {
       if (!attn_warp_wait(B, &B->item_full[n & 1], (n >> 1) & 1, ns, SITE_ATTN_SOFTMAX)) break;
       const AttnItem it = B->item[n & 1];
@@ -537,8 +541,10 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int ntk = it.packed >> 9;
       const int rows_total = it.packed & 0x1FF;
       const int nrows = x == 0 ? min(rows_total, Cfg::BM) : rows_total - Cfg::BM;
+      const bool pair = rows_total > Cfg::BM;   // both tiles present: take turns
       if (nrows <= 0) {          // this item has no tile B
         g += ntk;
+        other_before += ntk;     // tile A's steps of this item
         continue;
       }
       float m_ref = -INFINITY, l = 0.f;
@@ -553,10 +559,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         tc_fence_after();
         const uint32_t mk[4] = {B->meta[mi][0], B->meta[mi][1], B->meta[mi][2], B->meta[mi][3]};
         float sv[128];
-        tmem_ld128_sync(tmem + lane_off + Cfg::tm_s(x), sv);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B->s_free[x]);   // S buffer may be overwritten now
+        tmem_ld128_sync(s_addr, sv);
         ++n_s;
         // masked raw scores and the tile max; the mask is warp-uniform.  The
         // scale (into the log2 domain) is applied once to the max and folded
@@ -572,6 +575,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           for (int e = 0; e < 32; e += 2)
             mx4[(e >> 1) & 3] = max3f(mx4[(e >> 1) & 3], sv[c * 32 + e], sv[c * 32 + e + 1]);
         }
+        // wait for the turn: tile A's step t after tile B's step t-1, tile B's
+        // step t after tile A's step t
+        if (pair && (x == 1 || t > 0)) {
+          const uint32_t want = other_before + t - (x == 0 ? 1 : 0);   // index of the other's step
+          if (!attn_warp_wait(B, &B->exp_done[x ^ 1], want & 1, ns, SITE_ATTN_SOFTMAX)) {
+            ok = false;
+            break;
+          }
+        }
         const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         float alpha = 1.f;
         if (mt > m_ref + kRescaleLog2) {   // also taken on the first tile (m_ref = -inf)
@@ -586,46 +598,38 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 128; e += 2) {
           const float2 a2 = fma_f32x2(make_float2(sv[e], sv[e + 1]), sl2x2, nm2);
-          const float2 p2 = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+          float2 p2;
+          if ((e >> 1) % 64 < SVG_EXP_POLY_PAIRS)   // a share of the pairs on the FMA pipe
+            p2 = exp2_poly_x2(a2);
+          else
+            p2 = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
           rs2 = add_f32x2(rs2, p2);
-          packed[e >> 1] = pack_bf16x2(p2.x, p2.y);
+          packed[e >> 1] = SVG_PACK_INT ? pack_bf16x2_int(p2.x, p2.y) : pack_bf16x2(p2.x, p2.y);
         }
-        if (t >= 1) {  // PV_x(t-1) must be done before P_x and O_x are touched
-          if (!attn_warp_wait(B, &B->o_full[x], n_o & 1, ns, SITE_ATTN_SOFTMAX)) { ok = false; break; }
-          tc_fence_after();
-          ++n_o;
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {   // rescale O rows in TMEM
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->exp_done[x]);
+        // S_x(t) completing implies PV_x(t-1) completed (MMAs run in issue
+        // order), so O_x is stable here
+        if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {   // rescale O rows in TMEM
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float ov[32];
-              tmem_ld32_sync(o_addr + c * 32, ov);
+          for (int c = 0; c < D / 32; ++c) {
+            float ov[32];
+            tmem_ld32_sync(o_addr + c * 32, ov);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-              tmem_st32(o_addr + c * 32, ov);
-            }
-            tmem_st_wait();
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(o_addr + c * 32, ov);
           }
         }
         l = l * alpha + (rs2.x + rs2.y);
-        // P row: two 64-key halves, each one 128-byte swizzle row (K-major,
-        // 16-byte chunks XOR row % 8)
-#pragma unroll
-        for (int kh = 0; kh < 2; ++kh) {
-          uint8_t *prow = sPx + kh * Cfg::HALF_P + row * 128;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t chunk = u ^ (row & 7);
-            const int b = kh * 32 + 4 * u;
-            *reinterpret_cast<uint4 *>(prow + chunk * 16) =
-                make_uint4(packed[b], packed[b + 1], packed[b + 2], packed[b + 3]);
-          }
-        }
-        fence_proxy_async_smem();
+        // P row: 128 keys as 64 bf16 pairs over the first 64 columns of S_x
+        tmem_st64(s_addr, packed);
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B->p_full[x]);
       }
       if (!ok) break;
+      if (x == 1 || pair) other_before += ntk;   // the other tile's steps of this item
       if (!attn_warp_wait(B, &B->o_full[x], n_o & 1, ns, SITE_ATTN_SOFTMAX)) break;
       tc_fence_after();
       ++n_o;
@@ -713,21 +717,27 @@ __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
   ktiles[idx] = (slots + kSlotsPerTile - 1) / kSlotsPerTile;
 }
 
-// Single block: one AttnItem per 256 query rows, ordered by head group, then
-// by descending estimated cost inside a group (key tiles x query tiles; a
-// counting sort over kAttnBuckets buckets).  The attention kernel's CTAs
-// claim items in this order from a shared counter: a group's K/V (a few heads)
-// stays in L2 while its items run, and inside the group the longest items go
-// first (greedy list scheduling), so an SM that drew short items takes more
-// of them.  Also resets that counter.
+// Single block: one AttnItem per 256 query rows, in claiming order (a
+// counting sort over kAttnBuckets buckets of the estimated cost = key tiles x
+// query tiles).  Long items (cost >= kAttnBigCost: q-clusters whose centroid
+// scores are flat select most of the keys) come first, longest first across
+// all heads, so none of them starts late and sets the tail; the rest follow
+// by head group (a few heads, whose K/V stay in L2 while their items run),
+// longest first inside a group.  The attention kernel's CTAs claim items in
+// this order from a shared counter (greedy list scheduling), so an SM that
+// drew short items takes more of them.  Also resets that counter.
 constexpr int kAttnBuckets = 1024;
-constexpr int kAttnGroups = 16;                            // head groups
-constexpr int kAttnCostBuckets = kAttnBuckets / kAttnGroups;
+constexpr int kAttnBigCost = 32;
+constexpr int kAttnBigBuckets = 256;                       // costs 32 .. 287 and above
+constexpr int kAttnGroups = 16;                            // head groups of the short items
+constexpr int kAttnCostBuckets = (kAttnBuckets - kAttnBigBuckets) / kAttnGroups;   // 48 > kAttnBigCost
 
 __device__ __forceinline__ int attn_item_bucket(int h, int heads_per_group, int kt, int rows) {
   const int cost = kt * (rows > 128 ? 2 : 1);
+  if (cost >= kAttnBigCost)
+    return kAttnBigBuckets - 1 - min(cost - kAttnBigCost, kAttnBigBuckets - 1);
   const int grp = min(h / heads_per_group, kAttnGroups - 1);
-  return grp * kAttnCostBuckets + kAttnCostBuckets - 1 - min(cost, kAttnCostBuckets - 1);
+  return kAttnBigBuckets + grp * kAttnCostBuckets + kAttnCostBuckets - 1 - cost;
 }
 
 __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(

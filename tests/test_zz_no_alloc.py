@@ -11,12 +11,11 @@ contents when the second one runs).
 
 This file is named so that pytest collects it last.
 """
-import numpy as np
 import pytest
 import torch
 
 import synth
-from tests.helpers import ATTN_MAX_ABS, ATTN_REL_L2, check_attention, dev_bf16, dev_f32
+from tests.helpers import dev_bf16, dev_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -51,9 +50,10 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         got, got_lse = svg.sparse_attn_noalloc(*args, want_lse=True)
         torch.cuda.synchronize()
         assert svg.get_error() == 0
-        a, b = got.float().cpu().numpy(), ref.float().cpu().numpy()
-        check_attention(a, b, f"no-alloc vs workspace ({wl.name})")
-        assert np.max(np.abs(got_lse.cpu().numpy() - ref_lse.cpu().numpy())) < 1e-3
+        # the same kernel on the same inputs: every row is computed by one CTA
+        # over a fixed sequence of key tiles, so the results are bit-identical
+        assert torch.equal(got, ref), f"no-alloc vs workspace ({wl.name})"
+        assert torch.equal(got_lse, ref_lse), f"no-alloc vs workspace lse ({wl.name})"
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
