@@ -330,8 +330,9 @@ def run_svg(args, wl):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    if svg.get_error() != 0:
-        raise RuntimeError("device error word set during warm-up")
+    err = svg.get_error_detail()
+    if err[0] != 0:
+        raise RuntimeError("device error word set during warm-up: status %d at %s, CTA %d" % err)
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     if world > 1:
@@ -357,8 +358,9 @@ def run_svg(args, wl):
     if world > 1:
         torch.distributed.barrier()
     local_ms = t_start.elapsed_time(t_end)
-    if svg.get_error() != 0:
-        raise RuntimeError("device error word set during the timed steps")
+    err = svg.get_error_detail()
+    if err[0] != 0:
+        raise RuntimeError("device error word set during the timed steps: status %d at %s, CTA %d" % err)
     stage_ms = {n: statistics.mean(events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps))
                 for i, n in enumerate(stage_names)}
 

@@ -191,14 +191,14 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
  * is fixed when it starts, or a runtime that forbids device allocation after
  * initialisation.  This call takes the same inputs and outputs as
  * svg_sparse_attn and computes the same result, but its scratch space is a
- * fixed array compiled into the library (SVG_NOALLOC_SCRATCH_BYTES, 2 MiB) that
+ * fixed array compiled into the library (SVG_NOALLOC_SCRATCH_BYTES, 4 MiB) that
  * every GPU which loads the library holds until the process exits.
  *
  *  - Limit: svg_sparse_attn_workspace_size(BH, N, Cq), about
- *    16*BH*(ceil(N/256) + Cq) + 8*BH*Cq bytes, must not exceed
- *    SVG_NOALLOC_SCRATCH_BYTES (e.g. 80 heads x 75,600 tokens x 200 q-clusters
- *    needs 0.8 MB); larger sizes return SVG_ERR_WORKSPACE before anything is
- *    launched.
+ *    16*BH*(ceil(N/256) + Cq) + 8*BH*Cq bytes plus 2.5 MiB of per-CTA key
+ *    ranges, must not exceed SVG_NOALLOC_SCRATCH_BYTES (e.g. 80 heads x 75,600
+ *    tokens x 200 q-clusters needs 3.4 MB); larger sizes return
+ *    SVG_ERR_WORKSPACE before anything is launched.
  *  - It allocates and frees nothing (no cudaMalloc, no cudaFree, no
  *    allocating library routine).
  *  - The first call on each device looks up the device address of the array
@@ -209,7 +209,7 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
  *    clearing, but calls whose executions overlap on the GPU (different
  *    streams, or host threads) race on the array: order them on one stream.
  */
-#define SVG_NOALLOC_SCRATCH_BYTES (2u << 20)
+#define SVG_NOALLOC_SCRATCH_BYTES (4u << 20)
 svg_status svg_sparse_attn_noalloc(const void *qp, const void *kp, const void *vp, int BH, int N,
                                    int D, const int32_t *q_off, int Cq, const int32_t *k_off,
                                    int Ck, const int32_t *sel_count, const int32_t *sel_cols,
@@ -231,6 +231,28 @@ svg_status svg_unpermute(const void *xp, const int32_t *perm, int BH, int N, int
  */
 svg_status svg_get_error(svg_stream_t stream);
 void svg_set_wait_timeout_ns(uint64_t ns);
+
+/* Where the first recorded device error came from (the site field of the
+ * device error word). */
+typedef enum svg_error_site {
+  SVG_SITE_NONE = 0,
+  SVG_SITE_ATTN_PRODUCER = 1,   /* attention: item loader or TMA producer warp */
+  SVG_SITE_ATTN_MMA = 2,        /* attention: an MMA issuer warp */
+  SVG_SITE_ATTN_SOFTMAX = 3,    /* attention: a softmax warp */
+  SVG_SITE_ATTN_DRAIN = 4,      /* attention: waiting for copies in flight after an abort */
+  SVG_SITE_ATTN_EMPTY_ROW = 5,  /* attention planning: bad k-cluster id or no keys selected */
+  SVG_SITE_PERMUTE_RANGE = 6,   /* permute: cluster id outside [0, C) */
+  SVG_SITE_KMEANS_MMA = 7,      /* k-means assign: MMA issuer warp */
+  SVG_SITE_KMEANS_EPI = 8,      /* k-means assign: epilogue warps */
+  SVG_SITE_KMEANS_RANGE = 9,    /* k-means update: cluster id outside [0, C) */
+  SVG_SITE_KMEANS_DRAIN = 10    /* k-means assign: waiting for copies in flight after an abort */
+} svg_error_site;
+
+/* Same as svg_get_error (synchronises, returns and clears the error word),
+ * and also reports where the error came from: *site (an svg_error_site) and
+ * *block (the low 16 bits of the recording CTA's blockIdx.x); both 0 when
+ * nothing was recorded.  Either pointer may be NULL. */
+svg_status svg_get_error_detail(svg_stream_t stream, int32_t *site, int32_t *block);
 
 /* Test hook for failure detection (no GPU fault involved): fault = 1 makes
  * the following svg_sparse_attn launches skip loading their query tiles, so

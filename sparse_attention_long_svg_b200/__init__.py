@@ -38,6 +38,7 @@ SIGNATURES = {
     "svg_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
     "svg_debug_set_fault": (None, [_I]),
     "svg_get_error": (_I, [_P]),
+    "svg_get_error_detail": (_I, [_P, _P, _P]),
     "svg_kmeans_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "svg_kmeans": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "svg_permute_workspace_size": (_SZ, [_I, _I, _I]),
@@ -57,7 +58,7 @@ SIGNATURES = {
 
 PROFILE_KERNELS = {"kmeans_assign": 0, "sparse_attn": 1}
 
-NOALLOC_SCRATCH_BYTES = 2 << 20   # SVG_NOALLOC_SCRATCH_BYTES in include/svg.h
+NOALLOC_SCRATCH_BYTES = 4 << 20   # SVG_NOALLOC_SCRATCH_BYTES in include/svg.h
 
 _lib = None
 
@@ -121,6 +122,18 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 def get_error(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error word."""
     return load_library().svg_get_error(_stream(stream))
+
+
+ERROR_SITES = {0: "none", 1: "attention producer", 2: "attention MMA issuer", 3: "attention softmax",
+               4: "attention drain", 5: "attention planning", 6: "permute range", 7: "k-means MMA issuer",
+               8: "k-means epilogue", 9: "k-means range", 10: "k-means drain"}
+
+
+def get_error_detail(stream=None) -> Tuple[int, str, int]:
+    """Like get_error, also naming where the error was recorded: (status, site, CTA index)."""
+    site, block = ctypes.c_int32(), ctypes.c_int32()
+    st = load_library().svg_get_error_detail(_stream(stream), ctypes.byref(site), ctypes.byref(block))
+    return st, ERROR_SITES.get(site.value, str(site.value)), block.value
 
 
 def set_wait_timeout_ns(ns: int):

@@ -27,32 +27,28 @@
 //   warp 8     TMA producer: Q tiles; K and V tiles of every key tile into
 //              two rings (two slots each at D = 128)
 //   warps 9, 11 MMA issuers, one per query tile (warp 9 owns TMEM): the
-//              sequence S(0), PV(0), S(1), PV(1), ... with S_x = Q_x K^T (A and
-//              B in shared memory) and O_x += P_x V (A = P in tensor memory)
+//              sequence S(0), S(1), PV(0), S(2), PV(1), ... with S_x = Q_x K^T
+//              and O_x += P V (operands in shared memory)
 //   warp 10    item loader: claims the next item from a counter shared by all
 //              CTAs (list sorted by head group, then longest first), prefetches
 //              its query rows into L2, merges its key ranges into runs
 // Tensor memory per query tile x: S_x (128 fp32 columns) and O_x (D
-// columns).  The softmax reads S_x(t) into registers and writes P_x(t) as
-// bf16 pairs over the first 64 columns of S_x, where the PV MMA takes it as
-// its A operand; S_x(t+1) is issued after PV_x(t), and MMAs run in issue
-// order, so it overwrites P only after PV has read it.  The two query tiles
-// alternate on the tensor pipe: one tile's MMAs run while the other's
-// softmax computes.  O accumulates in TMEM across the item's key tiles; the
-// softmax warps rescale it in place only when a row's running max grows by
-// more than 2^8 (exact: every probability is taken against the same
-// reference max that O and the row sum use).
+// columns).  The softmax copies S_x(t) to registers and releases it at once,
+// so S_x(t+1) runs on the tensor cores while the softmax of step t computes.
+// The two query tiles take turns on their exponentials (the MUFU-bound part),
+// so one tile's exponentials overlap the other tile's MMAs; the turns also
+// let both tiles share one P buffer in shared memory (bf16, 128-byte
+// swizzled, K-major): P_x(t) is written once the previous PV (the other
+// tile's) has read it.  O accumulates in TMEM across the item's key tiles;
+// the softmax warps rescale it in place only when a row's running max grows
+// by more than 2^8 (exact: every probability is taken against the same
+// reference max that O and the row sum use).  The merged key ranges of the
+// CTA's next two items live in two global scratch slots of the workspace,
+// one per header slot.
 #pragma once
 #include "common.cuh"
 
 namespace svg {
-
-#ifndef SVG_EXP_POLY_PAIRS
-#define SVG_EXP_POLY_PAIRS 0
-#endif
-#ifndef SVG_PACK_INT
-#define SVG_PACK_INT 0
-#endif
 
 constexpr int kItemRows = 256;     // query rows per work item (two 128-row tiles)
 constexpr int kSlotsPerTile = 16;  // 8-row slots per 128-key tile
@@ -75,20 +71,23 @@ struct AttnCfg {
   static constexpr int KV_BYTES = BN * D * 2;         // one K or V tile
   static constexpr int HALF_Q = BM * 128;             // one 64-channel half of a Q tile
   static constexpr int HALF_KV = BN * 128;            // same for a K/V tile
+  static constexpr int P_BYTES = BM * BN * 2;         // the shared P tile
+  static constexpr int HALF_P = BM * 128;             // one 64-key half of it
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_P = OFF_Q + 2 * QT_BYTES;
+  static constexpr int OFF_K = OFF_P + P_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int MAX_SEL = 1024;                // selected k-clusters per q-cluster
-  static constexpr int OFF_RANGES = OFF_V + KST * KV_BYTES;   // int2 (first row, rows) per run
-  static constexpr int OFF_BAR = OFF_RANGES + MAX_SEL * 8;
+  static constexpr int OFF_BAR = OFF_V + KST * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers/meta + alignment slack
-  // TMEM: S (then P) of tile x at x*128 (128 columns); O of tile x at 256 + x*128
+  // TMEM: S of tile x at x*128 (128 columns); O of tile x at 256 + x*128
   static constexpr uint32_t TM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
   // warp 9 issues tile A's MMAs (and owns TMEM), warp 11 tile B's
   static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, LOADER_WARP = 10, MMA_B_WARP = 11;
   static constexpr int THREADS = 12 * 32;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   __device__ static constexpr uint32_t tm_s(int x) { return x * 128; }
   __device__ static constexpr uint32_t tm_o(int x) { return 256 + x * 128; }
 };
@@ -101,15 +100,6 @@ struct AttnMaps {
   CUtensorMap k[kNumBoxSizes];
   CUtensorMap v[kNumBoxSizes];
 };
-
-// Entry e of an item with n key tiles in the ring order K0, K1, V0, K2, V1,
-// ..., K(n-1), V(n-2), V(n-1): returns the key tile and sets is_k.
-__device__ __forceinline__ int attn_entry(int n, int e, bool &is_k) {
-  if (e == 0) { is_k = true; return 0; }
-  if (e == 2 * n - 1) { is_k = false; return n - 1; }
-  is_k = (e & 1) != 0;
-  return is_k ? (e + 1) >> 1 : (e >> 1) - 1;
-}
 
 // Sets bits [first, first + count) of a 128-bit mask held in four registers.
 __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count) {
@@ -126,18 +116,18 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int first, int count)
 }
 
 struct AttnBarriers {
-  uint64_t q_full, q_empty[2];                      // q_empty: [tile]
+  uint64_t q_full[2], q_empty[2];                   // [tile]
   uint64_t k_full[4], v_full[4];
   uint64_t k_empty[2][4], v_empty[2][4];            // [tile][slot]: released by that tile's MMAs
   uint64_t meta_full[kMetaRing];
-  uint64_t s_full[2], p_full[2], o_full[2];   // [tile]
-  uint64_t exp_done[2];                       // [tile]: its four softmax warps finished a step's exponentials
+  uint64_t s_full[2], s_free[2], p_full[2], o_full[2];   // [tile]
+  uint64_t p_free[2];                         // [tile]: a PV of that tile (reading P) has completed
   uint64_t item_full[2], item_empty[2];
-  uint64_t ranges_full, ranges_empty;
   uint64_t drain[2];
   AttnItem item[2];      // item header ring written by the loader warp
-  int32_t ranges_cnt;    // runs of the item whose ranges are in shared memory
+  int32_t ranges_cnt[2]; // merged runs of the item in header slot [b]
   uint32_t meta[kMetaRing][4];   // per key tile: 128-bit key validity mask
+  uint32_t exp_steps[2]; // [tile]: 4 x the steps whose exponentials that tile has finished (one add per warp)
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -151,6 +141,7 @@ struct AttnParams {
   float *lse;
   const int32_t *perm;   // optional: write row r of a head to row perm[r] (un-permuted output)
   unsigned long long *issued;   // optional: += (query tile, key tile) pairs issued
+  int2 *ranges;          // per CTA: 2 x MAX_SEL merged key runs (first row, rows), one slot per header slot
   int N, Cq, Ck, BH;
   float scale_log2;      // softmax scale * log2(e)
   uint64_t wait_ns;
@@ -186,6 +177,29 @@ __device__ __forceinline__ bool warp_aborted(AttnBarriers *b) {
   return __any_sync(0xffffffffu, aborted(b));
 }
 
+// Warp-wide wait until a shared-memory progress counter reaches `target`
+// (wrap-safe comparison); lane 0 polls, bounded like the barrier waits.
+__device__ __forceinline__ bool attn_warp_wait_count(AttnBarriers *b, const uint32_t *ctr, uint32_t target,
+                                                     uint64_t ns, uint32_t site) {
+  int ok = 1;
+  if (lane_id() == 0) {
+    const volatile uint32_t *c = ctr;
+    if (static_cast<int32_t>(*c - target) < 0) {
+      const long long t0 = clock64();
+      const long long limit = static_cast<long long>(ns) * 2;
+      while (static_cast<int32_t>(*c - target) < 0) {
+        if (clock64() - t0 > limit) {
+          ok = 0;
+          record_error(SVG_ERR_TIMEOUT, site);
+          atomicExch(&b->abort_flag, 1);
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Number of selected k-clusters of a block-list row, clamped to [0, limit];
 // a count outside that range is recorded as a device check failure.
 __device__ __forceinline__ int attn_sel_count(const int32_t *sel_count, size_t row, int limit) {
@@ -205,15 +219,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = smem + Cfg::OFF_Q;
+  uint8_t *sP = smem + Cfg::OFF_P;
   uint8_t *sK = smem + Cfg::OFF_K;
   uint8_t *sV = smem + Cfg::OFF_V;
-  int2 *sRanges = reinterpret_cast<int2 *>(smem + Cfg::OFF_RANGES);
+  int2 *gRanges = P.ranges + static_cast<size_t>(blockIdx.x) * 2 * Cfg::MAX_SEL;
   AttnBarriers *B = reinterpret_cast<AttnBarriers *>(smem + Cfg::OFF_BAR);
   const int warp = static_cast<int>(warp_id());
   const int lane = static_cast<int>(lane_id());
 
   if (threadIdx.x == 0) {
-    mbar_init(&B->q_full, 1);
     for (int s = 0; s < 4; ++s) {
       mbar_init(&B->k_full[s], 1);
       mbar_init(&B->v_full[s], 1);
@@ -225,16 +239,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     for (int s = 0; s < kMetaRing; ++s) mbar_init(&B->meta_full[s], 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&B->s_full[x], 1);
+      mbar_init(&B->s_free[x], 4);
       mbar_init(&B->p_full[x], 4);
-      mbar_init(&B->exp_done[x], 4);
+      mbar_init(&B->q_full[x], 1);
+      B->exp_steps[x] = 0;
       mbar_init(&B->o_full[x], 1);
       mbar_init(&B->item_full[x], 1);
       mbar_init(&B->item_empty[x], kItemReaders);
       mbar_init(&B->q_empty[x], 1);
       mbar_init(&B->drain[x], 1);
     }
-    mbar_init(&B->ranges_full, 1);
-    mbar_init(&B->ranges_empty, 1);
+    mbar_init(&B->p_free[0], 1);
+    mbar_init(&B->p_free[1], 1);
     B->abort_flag = 0;
     fence_mbar_init();
   }
@@ -260,8 +276,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     // ------------------------------------------------------------ item loader
     // Claims the next item of the list with an atomic counter, so an SM that
     // finishes early takes more work; after the last item it publishes an end
-    // marker (h = -1).  The key ranges have one shared-memory slot: the
-    // ranges of item n are written once the producer has finished item n-1.
+    // marker (h = -1).  The key ranges of item n go to the range slot of its
+    // header slot n & 1, free once every reader has released item n - 2 (the
+    // producer releases it after its last key tile).
     const int max_sel = min(P.Ck, Cfg::MAX_SEL);
     for (int n = 0;; ++n) {
       const int buf = n & 1;
@@ -287,158 +304,264 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int cnt = attn_sel_count(P.sel_count, row, max_sel);
       const int32_t *cols = P.sel_cols + row * P.Ck;
       const int32_t *koff = P.k_off + static_cast<size_t>(it.h) * (P.Ck + 1);
-      ok = true;
-      if (lane == 0 && n >= 1) ok = attn_wait(B, &B->ranges_empty, (n - 1) & 1, ns, SITE_ATTN_PRODUCER);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      for (int c = lane; c < cnt; c += 32) {
-        const int j = cols[c];
-        int2 r = make_int2(0, 0);  // out-of-range ids are flagged by the planning kernel
-        if (j >= 0 && j < P.Ck) {
-          r.x = koff[j];
-          r.y = koff[j + 1] - r.x;
-        }
-        sRanges[c] = r;
-      }
-      __syncwarp();
-      if (lane == 0) {   // merge touching ranges into runs (same rule as the planning kernel)
-        int m = 0, run_end = -1;
-        for (int c = 0; c < cnt; ++c) {
-          const int2 r = sRanges[c];
-          if (r.y <= 0) continue;
-          if (m > 0 && r.x == run_end) {
-            sRanges[m - 1].y += r.y;
-          } else {
-            sRanges[m++] = r;
+      // Merge touching ranges into runs (same rule as the planning kernel),
+      // 32 selected clusters at a time, one per lane: a non-empty range opens
+      // a run unless it starts where the previous non-empty range (in
+      // selection order) ended.  The open run is carried between chunks.
+      int2 *rng = gRanges + buf * Cfg::MAX_SEL;
+      int m = 0, open_x = 0, open_end = -1;   // runs opened so far; the open run
+      for (int c0 = 0; c0 < cnt; c0 += 32) {
+        const int c = c0 + lane;
+        int x = 0, len = 0;   // out-of-range ids are flagged by the planning kernel
+        if (c < cnt) {
+          const int j = cols[c];
+          if (j >= 0 && j < P.Ck) {
+            x = koff[j];
+            len = koff[j + 1] - x;
           }
-          run_end = r.x + r.y;
         }
-        B->ranges_cnt = m;
+        const bool valid = len > 0;
+        const int end = x + len;
+        const unsigned below_mask = (1u << lane) - 1u;
+        const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+        const unsigned vb = vmask & below_mask;
+        const int pv = vb ? 31 - __clz(vb) : 0;
+        const int pv_end = __shfl_sync(0xffffffffu, end, pv);
+        const int prev_end = vb ? pv_end : open_end;   // end of the previous non-empty range
+        const bool opens = valid && x != prev_end;
+        const unsigned smask = __ballot_sync(0xffffffffu, opens);
+        const unsigned sb = smask & below_mask;
+        const int ps = sb ? 31 - __clz(sb) : 0;
+        const int ps_x = __shfl_sync(0xffffffffu, x, ps);
+        if (opens) {   // close the previous run: it ends at prev_end
+          const int idx = m + __popc(sb);
+          const int run_x = sb ? ps_x : open_x;
+          if (idx > 0) rng[idx - 1] = make_int2(run_x, prev_end - run_x);
+        }
+        if (smask) open_x = __shfl_sync(0xffffffffu, x, 31 - __clz(smask));
+        if (vmask) open_end = __shfl_sync(0xffffffffu, end, 31 - __clz(vmask));
+        m += __popc(smask);
+      }
+      if (lane == 0) {
+        if (m > 0) rng[m - 1] = make_int2(open_x, open_end - open_x);
+        __threadfence_block();
+        B->ranges_cnt[buf] = m;
         B->item[buf] = it;
         __threadfence_block();
-        mbar_arrive(&B->ranges_full);
         mbar_arrive(&B->item_full[buf]);
       }
       __syncwarp();
     }
   } else if (warp == Cfg::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
-    // Per item: the Q tiles, then K(t) and V(t) of every key tile t (both
-    // through the same box list).  K(t + KST) waits for S(t) of both query
-    // tiles, V(t + KST) for PV(t).
-    uint32_t g = 0;         // global key-tile counter
-    uint32_t nq = 0;        // Q loads issued (for the drain)
-    uint32_t gk = 0, gv = 0;   // K and V tiles issued (for the drain)
+    // Two streams, issued by one thread that polls both: the K side takes the
+    // items in order (Q tiles, then K(t) of every key tile t, cutting each
+    // tile into boxes), the V side issues V(t) from the same box list.  Each
+    // load is issued as soon as its ring slot is free: K(t + KST) once both
+    // present query tiles' S(t) are done, V(t + KST) once their PV(t) are, so
+    // a slot held by the slower tile never holds up the other ring.  Box
+    // lists of key tiles whose V is not yet issued stay in a small ring.
     // A slot (and Q) is reused once every query tile of its last occupant has
     // released it: tile A is in every item, tile B only in items of > 128
-    // rows; slot_b[s] = whether the slot's last occupant had tile B,
-    // rel_b[s] / nq_b = tile-B releases of the slot / of Q expected so far.
-    bool slot_b[4] = {false, false, false, false}, prev_b = false;
-    uint32_t rel_b[4] = {0, 0, 0, 0}, nq_b = 0;
-    if (lane == 0) {
-      bool ok = true;
-      for (int n = 0; ok && !aborted(B); ++n) {
-        const int buf = n & 1;
-        if (!attn_wait(B, &B->item_full[buf], (n >> 1) & 1, ns, SITE_ATTN_PRODUCER)) break;
-        const AttnItem it = B->item[buf];
-        if (it.h < 0) {                     // end of the list
-          mbar_arrive(&B->item_empty[buf]);
-          break;
-        }
-        if (!attn_wait(B, &B->ranges_full, n & 1, ns, SITE_ATTN_PRODUCER)) break;
-        const int cnt = B->ranges_cnt;
-        const int ntk = it.packed >> 9;
-        const bool has_b = (it.packed & 0x1FF) > Cfg::BM;
-        if (n > 0 && (!attn_wait(B, &B->q_empty[0], (n - 1) & 1, ns, SITE_ATTN_PRODUCER) ||
-                      (prev_b && !attn_wait(B, &B->q_empty[1], (nq_b - 1) & 1, ns, SITE_ATTN_PRODUCER))))
-          break;
-        prev_b = has_b;
-        if (has_b) ++nq_b;
-        if (P.fault != 1) {
-          mbar_arrive_expect_tx(&B->q_full, Cfg::QT_BYTES * (has_b ? 2 : 1));
-          const int qrow = it.h * P.N + it.q0;
+    // rows; slot_b[r][s] = whether slot s of ring r (0 = K, 1 = V) last held a
+    // tile with tile B, rel_b[r][s] / nq_b = tile-B releases expected so far.
+    // The whole warp runs the loop with identical control flow (barrier tests
+    // are made by lane 0 and broadcast); lane 0 issues the arrivals and the
+    // Q copies, lane b the copies of box b of a key tile.  Key ranges are
+    // read 32 at a time into a register window; every other piece of state
+    // is in registers (no local memory).
+    constexpr int kBoxRing = Cfg::KST + 2;   // box lists of tiles whose V is not yet issued
+    auto test = [&](uint64_t *bar, uint32_t parity) {
+      return __shfl_sync(0xffffffffu, lane == 0 ? (mbar_test(bar, parity) ? 1 : 0) : 0, 0) != 0;
+    };
+    int2 win = make_int2(0, 0);
+    int win_base = -1;
+    const int2 *rng = gRanges;
+    {
+      // bit 4r + s: slot s of ring r last held a tile with tile B / parity of
+      // the tile-B releases of that slot expected so far
+      uint32_t slot_b = 0, rel_b = 0, nq_b = 0;
+      uint32_t tile_b = 0;               // bit e: box-ring entry e has tile B
+      int box_row[kBoxRing], box_code[kBoxRing];   // this lane's box of each entry: row, kind | slot << 8 (-1: none)
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (x == 1 && !has_b) break;
+      for (int e = 0; e < kBoxRing; ++e) box_row[e] = box_code[e] = -1;
+      uint32_t gk = 0, gv = 0, nq = 0, nq1 = 0;   // K and V tiles issued, Q loads issued (all, tile B)
+      int n = 0;                         // next item (header slot n & 1)
+      bool k_active = false, k_done = false, prev_b = false;
+      AttnItem it{};
+      int ntk = 0, tk = 0, cnt = 0, ci = 0, cur = 0, left = 0;
+      bool has_b = false;
+      const long long limit = static_cast<long long>(ns) * 2;
+      long long t_last = clock64();
+      while (!(k_done && gv == gk)) {
+        bool progress = false;
+        // ---- K side: start the next item
+        if (!k_active && !k_done && test(&B->item_full[n & 1], (n >> 1) & 1)) {
+          it = B->item[n & 1];
+          if (it.h < 0) {                   // end of the list
+            if (lane == 0) mbar_arrive(&B->item_empty[n & 1]);
+            k_done = true;
+            progress = true;
+          } else if ((n == 0 || (test(&B->q_empty[0], (n - 1) & 1) &&
+                                 (!prev_b || test(&B->q_empty[1], (nq_b - 1) & 1))))) {
+            cnt = B->ranges_cnt[n & 1];
+            rng = gRanges + (n & 1) * Cfg::MAX_SEL;
+            ntk = it.packed >> 9;
+            has_b = (it.packed & 0x1FF) > Cfg::BM;
+            prev_b = has_b;
+            if (has_b) ++nq_b;
+            if (P.fault != 1 && lane == 0) {
+              const int qrow = it.h * P.N + it.q0;
 #pragma unroll
-            for (int dh = 0; dh < Cfg::DH; ++dh)
-              tma_load_2d(sQ + x * Cfg::QT_BYTES + dh * Cfg::HALF_Q, &maps.q, dh * 64,
-                          qrow + x * Cfg::BM, &B->q_full);
+              for (int x = 0; x < 2; ++x) {
+                if (x == 1 && !has_b) break;
+                mbar_arrive_expect_tx(&B->q_full[x], Cfg::QT_BYTES);
+#pragma unroll
+                for (int dh = 0; dh < Cfg::DH; ++dh)
+                  tma_load_2d(sQ + x * Cfg::QT_BYTES + dh * Cfg::HALF_Q, &maps.q, dh * 64,
+                              qrow + x * Cfg::BM, &B->q_full[x]);
+              }
+            }
+            if (P.fault != 1) {
+              ++nq;
+              if (has_b) ++nq1;
+            }
+            tk = 0;
+            win_base = -1;
+            ci = cur = left = 0;
+            k_active = true;
+            progress = true;
           }
-          ++nq;
         }
-        int ci = 0, cur = 0, left = 0;
-        const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
-        for (int t = 0; t < ntk && ok; ++t, ++g) {
-          // cut tile t into boxes of 1..16 slots (8..128 rows): the largest
-          // power of two that fits both the tile and the rest of the run
-          int box_row[Cfg::NSLOT], box_kind[Cfg::NSLOT], nb = 0;
-          uint32_t mask[4] = {0, 0, 0, 0};
-          int sl = 0;
-          while (sl < Cfg::NSLOT) {
-            while (left <= 0 && ci < cnt) {
-              const int2 r = sRanges[ci++];
-              cur = r.x;
-              left = r.y;
+        // ---- K side: the next key tile of the item
+        if (k_active && gk - gv < static_cast<uint32_t>(kBoxRing)) {
+          const int slot = static_cast<int>(gk % Cfg::KST);
+          const uint32_t sbit = 1u << slot;
+          const bool free_slot =
+              gk < static_cast<uint32_t>(Cfg::KST) ||
+              (test(&B->k_empty[0][slot], ((gk / Cfg::KST) - 1) & 1) &&
+               (!(slot_b & sbit) || test(&B->k_empty[1][slot], (rel_b & sbit) ? 0u : 1u)));
+          if (free_slot) {
+            // cut the tile into boxes of 1..16 slots (8..128 rows): the largest
+            // power of two that fits both the tile and the rest of the run
+            const int rb = static_cast<int>(gk % kBoxRing);
+            const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
+            uint32_t mask[4] = {0, 0, 0, 0};
+            int sl = 0, nb = 0, my_row = -1, my_code = -1;
+            while (sl < Cfg::NSLOT) {
+              while (left <= 0 && ci < cnt) {
+                if ((ci & ~31) != win_base) {   // refill the window: ranges [ci & ~31, +32)
+                  win_base = ci & ~31;
+                  win = win_base + lane < cnt ? __ldcg(rng + win_base + lane) : make_int2(0, 0);
+                }
+                cur = __shfl_sync(0xffffffffu, win.x, ci & 31);
+                left = __shfl_sync(0xffffffffu, win.y, ci & 31);
+                ++ci;
+              }
+              const int space = Cfg::NSLOT - sl;
+              const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
+              int kind = 0;
+              while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
+              const int nsl = 1 << kind;
+              if (lane == nb) {
+                my_row = left > 0 ? it.h * P.N + cur : pad_row;
+                my_code = kind | (sl << 8);
+              }
+              if (left > 0) {
+                set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
+                cur += nsl * Cfg::SLOT;
+                left -= nsl * Cfg::SLOT;
+              }
+              ++nb;
+              sl += nsl;
             }
-            const int space = Cfg::NSLOT - sl;
-            const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
-            int kind = 0;
-            while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
-            const int nsl = 1 << kind;
-            if (left > 0) {
-              set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
-              box_row[nb] = it.h * P.N + cur;
-              cur += nsl * Cfg::SLOT;
-              left -= nsl * Cfg::SLOT;
-            } else {
-              box_row[nb] = pad_row;   // no keys left: finite filler rows, masked out
-            }
-            box_kind[nb] = kind | (sl << 8);
-            ++nb;
-            sl += nsl;
-          }
-          if (t == ntk - 1) mbar_arrive(&B->ranges_empty);   // the ranges are no longer read
-          const int mi = static_cast<int>(g % kMetaRing);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
-          mbar_arrive(&B->meta_full[mi]);
-          const int slot = static_cast<int>(g % Cfg::KST);
-          const uint32_t ph = ((g / Cfg::KST) - 1) & 1;
-          const bool reuse_b = g >= static_cast<uint32_t>(Cfg::KST) && slot_b[slot];
-          const uint32_t ph_b = (rel_b[slot] - 1) & 1;
-#pragma unroll
-          for (int kv = 0; kv < 2; ++kv) {     // K(t), then V(t)
-            uint64_t *full = kv ? &B->v_full[slot] : &B->k_full[slot];
-            if (g >= static_cast<uint32_t>(Cfg::KST) &&
-                (!attn_wait(B, kv ? &B->v_empty[0][slot] : &B->k_empty[0][slot], ph, ns, SITE_ATTN_PRODUCER) ||
-                 (reuse_b && !attn_wait(B, kv ? &B->v_empty[1][slot] : &B->k_empty[1][slot], ph_b, ns,
-                                        SITE_ATTN_PRODUCER)))) {
-              ok = false;
-              break;
+            for (int e = 0; e < kBoxRing; ++e) {
+              if (e == rb) {
+                box_row[e] = my_row;
+                box_code[e] = my_code;
+              }
             }
-            mbar_arrive_expect_tx(full, Cfg::KV_BYTES);
-            uint8_t *dst = (kv ? sV : sK) + slot * Cfg::KV_BYTES;
-            const CUtensorMap *maps_t = kv ? maps.v : maps.k;
-            for (int bx = 0; bx < nb; ++bx) {
-              const int kind = box_kind[bx] & 0xFF, at = box_kind[bx] >> 8;
+            tile_b = has_b ? (tile_b | (1u << rb)) : (tile_b & ~(1u << rb));
+            const int mi = static_cast<int>(gk % kMetaRing);
+            slot_b = has_b ? (slot_b | sbit) : (slot_b & ~sbit);
+            if (has_b) rel_b ^= sbit;
+            if (lane == 0) {
+#pragma unroll
+              for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
+              mbar_arrive(&B->meta_full[mi]);
+              mbar_arrive_expect_tx(&B->k_full[slot], Cfg::KV_BYTES);
+            }
+            __syncwarp();
+            if (my_code >= 0) {
+              const int kind = my_code & 0xFF, at = my_code >> 8;
 #pragma unroll
               for (int dh = 0; dh < Cfg::DH; ++dh)
-                tma_load_2d(dst + dh * Cfg::HALF_KV + at * 1024, &maps_t[kind], dh * 64, box_row[bx], full);
+                tma_load_2d(sK + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64,
+                            my_row, &B->k_full[slot]);
             }
-            if (kv)
-              gv = g + 1;
-            else
-              gk = g + 1;
+            ++gk;
+            progress = true;
+            if (++tk == ntk) {             // the item's ranges and header are no longer read
+              if (lane == 0) {
+                mbar_arrive(&B->item_empty[n & 1]);
+              }
+              ++n;
+              k_active = false;
+            }
           }
-          slot_b[slot] = has_b;
-          if (has_b) ++rel_b[slot];
         }
-        mbar_arrive(&B->item_empty[buf]);
+        // ---- V side
+        if (gv < gk) {
+          const int slot = static_cast<int>(gv % Cfg::KST);
+          const uint32_t sbit = 1u << (4 + slot);
+          const bool free_slot =
+              gv < static_cast<uint32_t>(Cfg::KST) ||
+              (test(&B->v_empty[0][slot], ((gv / Cfg::KST) - 1) & 1) &&
+               (!(slot_b & sbit) || test(&B->v_empty[1][slot], (rel_b & sbit) ? 0u : 1u)));
+          if (free_slot) {
+            const int rb = static_cast<int>(gv % kBoxRing);
+            const bool tb = (tile_b >> rb) & 1u;
+            slot_b = tb ? (slot_b | sbit) : (slot_b & ~sbit);
+            if (tb) rel_b ^= sbit;
+            int my_row = -1, my_code = -1;
+#pragma unroll
+            for (int e = 0; e < kBoxRing; ++e) {
+              if (e == rb) {
+                my_row = box_row[e];
+                my_code = box_code[e];
+              }
+            }
+            if (lane == 0) mbar_arrive_expect_tx(&B->v_full[slot], Cfg::KV_BYTES);
+            __syncwarp();
+            if (my_code >= 0) {
+              const int kind = my_code & 0xFF, at = my_code >> 8;
+#pragma unroll
+              for (int dh = 0; dh < Cfg::DH; ++dh)
+                tma_load_2d(sV + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64,
+                            my_row, &B->v_full[slot]);
+            }
+            ++gv;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (__shfl_sync(0xffffffffu, clock64() - t_last > limit ? 1 : 0, 0)) {
+          if (lane == 0) {
+            record_error(SVG_ERR_TIMEOUT, SITE_ATTN_PRODUCER);
+            atomicExch(&B->abort_flag, 1);
+          }
+          break;
+        } else if (warp_aborted(B)) {
+          break;
+        }
       }
       // drain: every load issued above lands on a full barrier; wait for the
       // last phase of each so no copy is in flight when the CTA exits.
-      if (aborted(B)) {
-        if (nq > 0) mbar_wait(&B->q_full, (nq - 1) & 1, 1000000000ull);
+      if (lane == 0 && aborted(B)) {
+        if (nq > 0) mbar_wait(&B->q_full[0], (nq - 1) & 1, 1000000000ull);
+        if (nq1 > 0) mbar_wait(&B->q_full[1], (nq1 - 1) & 1, 1000000000ull);
         for (uint32_t k = (gk >= static_cast<uint32_t>(Cfg::KST) ? gk - Cfg::KST : 0); k < gk; ++k)
           mbar_wait(&B->k_full[k % Cfg::KST], (k / Cfg::KST) & 1, 1000000000ull);
         for (uint32_t k = (gv >= static_cast<uint32_t>(Cfg::KST) ? gv - Cfg::KST : 0); k < gv; ++k)
@@ -447,18 +570,26 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     }
   } else if (warp == Cfg::MMA_WARP || warp == Cfg::MMA_B_WARP) {
     // ------------------------------------------------------------ MMA issuers
-    // One thread per query tile x issues that tile's sequence S(0), PV(0),
-    // S(1), PV(1), ... of every item that has the tile: S_x(t) once K(t) (and
-    // Q) has landed, PV_x(t) once the softmax has written P_x(t) and V(t) has
+    // One thread per query tile x issues that tile's chains for every item
+    // that has the tile, in the order S(0), S(1), PV(0), S(2), PV(1), ...:
+    // S_x(t) once K(t) (and Q) has landed and the softmax has read S_x(t-1)
+    // out of TMEM; PV_x(t) once the softmax has written P_x(t) and V(t) has
     // landed.  It releases each K/V slot and Q for its own tile; the producer
-    // reuses them when every present tile has released them.  Two issuers let
-    // one tile's chain queue on the tensor pipe while the other's executes.
+    // reuses them when every present tile has released them.  With two
+    // issuers one tile's chain queues on the tensor pipe while the other's
+    // executes.  Tile B skips items without tile B, yet its parity waits on
+    // the shared K/V slot barriers cannot pass on an older phase: its Q tile
+    // of an item (own barrier, one phase per tile-B item) is loaded only
+    // after tile A's last S of the previous item, so every earlier K tile has
+    // landed, and its first P write of the item waits for tile A's first PV
+    // of the item, so every earlier V tile has landed.
     const int x = warp == Cfg::MMA_WARP ? 0 : 1;
     if (lane == 0) {
       const SmemDesc qd = make_desc_sw128(smem_u32(sQ) + x * Cfg::QT_BYTES, 16, 1024);
+      const SmemDesc pd = make_desc_sw128(smem_u32(sP), 16, 1024);
       const SmemDesc kd0 = make_desc_sw128(smem_u32(sK), 16, 1024);
       const SmemDesc vd0 = make_desc_sw128(smem_u32(sV), Cfg::HALF_KV, 1024);
-      uint32_t g0 = 0, n_pv = 0;   // key tiles of earlier items; PV chains issued
+      uint32_t g0 = 0, n_s = 0, n_pv = 0, n_q = 0;   // key tiles of earlier items; S, PV chains issued; Q tiles used
       unsigned long long pairs = 0;
       for (uint32_t n = 0; !aborted(B); ++n) {
         if (!attn_wait(B, &B->item_full[n & 1], (n >> 1) & 1, ns, SITE_ATTN_MMA)) break;
@@ -470,35 +601,48 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           g0 += ntk;
           continue;
         }
-        if (!attn_wait(B, &B->q_full, n & 1, ns, SITE_ATTN_MMA)) break;
+        if (!attn_wait(B, &B->q_full[x], n_q & 1, ns, SITE_ATTN_MMA)) break;
+        ++n_q;
         bool ok = true;
-        for (int t = 0; t < ntk && ok; ++t) {
+        // op 2t issues S(t + 1) (S(0) before the loop), op 2t + 1 issues PV(t)
+        for (int op = -1; op < 2 * ntk && ok; ++op) {
+          const bool is_s = op < 0 || (op & 1) == 0;
+          const int t = op < 0 ? 0 : (is_s ? (op >> 1) + 1 : op >> 1);
+          if (is_s && t >= ntk) continue;
           const uint32_t gt = g0 + t;
           const int slot = static_cast<int>(gt % Cfg::KST);
           const uint32_t ph = (gt / Cfg::KST) & 1;
           const uint32_t slot_off = (slot * Cfg::KV_BYTES) >> 4;
-          if (!attn_wait(B, &B->k_full[slot], ph, ns, SITE_ATTN_MMA)) { ok = false; break; }
-          tc_fence_after();
-          mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
-              tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
-          mma_commit(&B->s_full[x]);
-          mma_commit(&B->k_empty[x][slot]);
-          if (t == ntk - 1) mma_commit(&B->q_empty[x]);   // the item's last S: Q may be replaced
-          if (!attn_wait(B, &B->p_full[x], n_pv & 1, ns, SITE_ATTN_MMA) ||
-              !attn_wait(B, &B->v_full[slot], ph, ns, SITE_ATTN_MMA)) {
-            ok = false;
-            break;
+          if (is_s) {
+            if (!attn_wait(B, &B->k_full[slot], ph, ns, SITE_ATTN_MMA) ||
+                (n_s > 0 && !attn_wait(B, &B->s_free[x], (n_s - 1) & 1, ns, SITE_ATTN_MMA))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
+                tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
+            mma_commit(&B->s_full[x]);
+            mma_commit(&B->k_empty[x][slot]);
+            if (t == ntk - 1) mma_commit(&B->q_empty[x]);   // the item's last S: Q may be replaced
+            ++n_s;
+          } else {
+            if (!attn_wait(B, &B->p_full[x], n_pv & 1, ns, SITE_ATTN_MMA) ||
+                !attn_wait(B, &B->v_full[slot], ph, ns, SITE_ATTN_MMA)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // A = P [128 q x 128 keys], K-major in two 64-key halves; B = V [128 keys x D],
+            // MN-major, 16 keys = 2048 bytes per K-step
+            mma_chain<Cfg::BN / 16, Cfg::HALF_P, 32, 4 * 2048, 2048>(
+                tmem + Cfg::tm_o(x), pd, SmemDesc{vd0.lo + slot_off, vd0.hi}, Cfg::IDESC_PV, t > 0 ? 1u : 0u);
+            mma_commit(&B->p_free[x]);                     // the shared P buffer may be rewritten
+            if (t == ntk - 1) mma_commit(&B->o_full[x]);   // the item's O of tile x is final
+            mma_commit(&B->v_empty[x][slot]);
+            ++n_pv;
+            ++pairs;
           }
-          tc_fence_after();
-          // A = P_x [128 q x 128 keys] in TMEM (the first 64 columns of S_x);
-          // B = V [128 keys x D], MN-major, 16 keys = 2048 bytes per K-step
-          mma_chain_ts<Cfg::BN / 16, 4 * 2048, 2048>(tmem + Cfg::tm_o(x), tmem + Cfg::tm_s(x),
-                                                     SmemDesc{vd0.lo + slot_off, vd0.hi}, Cfg::IDESC_PV,
-                                                     t > 0 ? 1u : 0u);
-          if (t == ntk - 1) mma_commit(&B->o_full[x]);   // the item's O of tile x is final
-          mma_commit(&B->v_empty[x][slot]);
-          ++n_pv;
-          ++pairs;
         }
         if (!ok) break;
         g0 += ntk;
@@ -523,15 +667,26 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const uint32_t s_addr = tmem + lane_off + Cfg::tm_s(x);
     const float sl2 = P.scale_log2;
     uint32_t g = 0, n_s = 0, n_o = 0;
-    // Exponentials take turns between the two tiles of an item (A(t), B(t),
-    // A(t+1), ...), so one tile's exponentials overlap the other tile's MMAs
-    // instead of competing for the same MUFU units.  exp_done[y] completes
-    // once per step of tile y; other_before counts the other tile's steps in
-    // earlier items (tile A runs every item, tile B only items of > 128 rows).
-    // Neither tile can get two completions ahead of the other's wait: tile B
-    // waits for A(t) before finishing B(t), A waits for B(t-1) before A(t),
-    // and an item's first S is issued only after both tiles' last PV.
+    // Exponentials take turns between the two tiles (A(t), B(t), A(t+1), ...),
+    // so one tile's exponentials overlap the other tile's MMAs instead of
+    // competing for the same MUFU units: B(t) starts once A has finished t+1
+    // steps of the item, A(t) once B has finished all its steps before B(t)
+    // (in an item without tile B: all of B's steps so far).  Progress is a
+    // monotonic counter per tile (exp_steps, 4 per step), not a barrier
+    // parity, because tile B skips items and a parity would alias once one
+    // tile runs two steps ahead of the other's wait.  other_before counts the
+    // other tile's steps in earlier items (tile A runs every item, tile B
+    // only items of > 128 rows).
     uint32_t other_before = 0;
+    // P writes to the shared buffer happen in the order A(0), B(0), A(1), ...
+    // (A(0), A(1), ... in items without tile B).  A write waits for the PV of
+    // the previous write, on the p_free barrier of the tile that made it, by
+    // that tile's PV count: pv_before[y] = PVs of tile y in earlier items.  A
+    // waiter is never two completions behind on that barrier (the previous PV
+    // of the same tile finished before the write that preceded ours), so the
+    // phase parity cannot alias.
+    uint32_t pv_before[2] = {0, 0};
+    bool have_prev = false, prev_pair = false;
     for (uint32_t n = 0; !warp_aborted(B); ++n) {
       if (!attn_warp_wait(B, &B->item_full[n & 1], (n >> 1) & 1, ns, SITE_ATTN_SOFTMAX)) break;
       const AttnItem it = B->item[n & 1];
@@ -545,6 +700,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       if (nrows <= 0) {          // this item has no tile B
         g += ntk;
         other_before += ntk;     // tile A's steps of this item
+        pv_before[0] += ntk;     // and its PVs
+        have_prev = true;
+        prev_pair = false;
         continue;
       }
       float m_ref = -INFINITY, l = 0.f;
@@ -560,6 +718,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         const uint32_t mk[4] = {B->meta[mi][0], B->meta[mi][1], B->meta[mi][2], B->meta[mi][3]};
         float sv[128];
         tmem_ld128_sync(s_addr, sv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B->s_free[x]);   // S_x(t + 1) may overwrite the buffer
         ++n_s;
         // masked raw scores and the tile max; the mask is warp-uniform.  The
         // scale (into the log2 domain) is applied once to the max and folded
@@ -575,11 +736,11 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           for (int e = 0; e < 32; e += 2)
             mx4[(e >> 1) & 3] = max3f(mx4[(e >> 1) & 3], sv[c * 32 + e], sv[c * 32 + e + 1]);
         }
-        // wait for the turn: tile A's step t after tile B's step t-1, tile B's
-        // step t after tile A's step t
-        if (pair && (x == 1 || t > 0)) {
-          const uint32_t want = other_before + t - (x == 0 ? 1 : 0);   // index of the other's step
-          if (!attn_warp_wait(B, &B->exp_done[x ^ 1], want & 1, ns, SITE_ATTN_SOFTMAX)) {
+        // wait for the turn: tile B's step t after tile A's step t, tile A's
+        // step t after tile B's step t-1 (or B's last step of earlier items)
+        {
+          const uint32_t want = x == 1 ? other_before + t + 1 : other_before + (pair ? t : 0);
+          if (want > 0 && !attn_warp_wait_count(B, &B->exp_steps[x ^ 1], 4u * want, ns, SITE_ATTN_SOFTMAX)) {
             ok = false;
             break;
           }
@@ -598,18 +759,32 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 128; e += 2) {
           const float2 a2 = fma_f32x2(make_float2(sv[e], sv[e + 1]), sl2x2, nm2);
-          float2 p2;
-          if ((e >> 1) % 64 < SVG_EXP_POLY_PAIRS)   // a share of the pairs on the FMA pipe
-            p2 = exp2_poly_x2(a2);
-          else
-            p2 = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+          const float2 p2 = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
           rs2 = add_f32x2(rs2, p2);
-          packed[e >> 1] = SVG_PACK_INT ? pack_bf16x2_int(p2.x, p2.y) : pack_bf16x2(p2.x, p2.y);
+          packed[e >> 1] = pack_bf16x2(p2.x, p2.y);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B->exp_done[x]);
-        // S_x(t) completing implies PV_x(t-1) completed (MMAs run in issue
-        // order), so O_x is stable here
+        if (lane == 0) atomicAdd(&B->exp_steps[x], 1u);
+        // the shared P buffer is free once the PV of the previous write has
+        // completed; that PV was issued after PV_x(t - 1) completed, so O_x
+        // is stable too
+        int py = -1;              // tile whose PV read P last, and that PV's index
+        uint32_t pidx = 0;
+        if (x == 1) {
+          py = 0;
+          pidx = pv_before[0] + t;                          // A(t)
+        } else if (t > 0) {
+          py = pair ? 1 : 0;
+          pidx = pv_before[py] + t - 1;                     // B(t-1), or A(t-1)
+        } else if (have_prev) {
+          py = prev_pair ? 1 : 0;
+          pidx = pv_before[py] - 1;                         // the previous item's last write
+        }
+        if (py >= 0 && !attn_warp_wait(B, &B->p_free[py], pidx & 1, ns, SITE_ATTN_SOFTMAX)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {   // rescale O rows in TMEM
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -621,15 +796,31 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
         l = l * alpha + (rs2.x + rs2.y);
-        // P row: 128 keys as 64 bf16 pairs over the first 64 columns of S_x
-        tmem_st64(s_addr, packed);
-        tmem_st_wait();
+        // P row: two 64-key halves, each one 128-byte swizzle row (K-major,
+        // 16-byte chunks XOR row % 8)
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+          uint8_t *prow = sP + kh * Cfg::HALF_P + row * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t chunk = u ^ (row & 7);
+            const int b = kh * 32 + 4 * u;
+            *reinterpret_cast<uint4 *>(prow + chunk * 16) =
+                make_uint4(packed[b], packed[b + 1], packed[b + 2], packed[b + 3]);
+          }
+        }
+        tmem_st_wait();           // O rescale stores (if any) have landed
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&B->p_full[x]);
       }
       if (!ok) break;
       if (x == 1 || pair) other_before += ntk;   // the other tile's steps of this item
+      pv_before[0] += ntk;
+      if (pair) pv_before[1] += ntk;
+      have_prev = true;
+      prev_pair = pair;
       if (!attn_warp_wait(B, &B->o_full[x], n_o & 1, ns, SITE_ATTN_SOFTMAX)) break;
       tc_fence_after();
       ++n_o;

@@ -19,18 +19,19 @@ namespace svg {
 // Layout: bits 0-7 status, bits 8-15 site id, bits 16-31 block index (low bits).
 __device__ uint32_t g_error_word = 0;
 
+// Site ids are the public svg_error_site values.
 enum ErrorSite : uint32_t {
-  SITE_NONE = 0,
-  SITE_ATTN_PRODUCER = 1,
-  SITE_ATTN_MMA = 2,
-  SITE_ATTN_SOFTMAX = 3,
-  SITE_ATTN_DRAIN = 4,
-  SITE_ATTN_EMPTY_ROW = 5,
-  SITE_PERMUTE_RANGE = 6,
-  SITE_KMEANS_MMA = 7,
-  SITE_KMEANS_EPI = 8,
-  SITE_KMEANS_RANGE = 9,
-  SITE_KMEANS_DRAIN = 10,
+  SITE_NONE = SVG_SITE_NONE,
+  SITE_ATTN_PRODUCER = SVG_SITE_ATTN_PRODUCER,
+  SITE_ATTN_MMA = SVG_SITE_ATTN_MMA,
+  SITE_ATTN_SOFTMAX = SVG_SITE_ATTN_SOFTMAX,
+  SITE_ATTN_DRAIN = SVG_SITE_ATTN_DRAIN,
+  SITE_ATTN_EMPTY_ROW = SVG_SITE_ATTN_EMPTY_ROW,
+  SITE_PERMUTE_RANGE = SVG_SITE_PERMUTE_RANGE,
+  SITE_KMEANS_MMA = SVG_SITE_KMEANS_MMA,
+  SITE_KMEANS_EPI = SVG_SITE_KMEANS_EPI,
+  SITE_KMEANS_RANGE = SVG_SITE_KMEANS_RANGE,
+  SITE_KMEANS_DRAIN = SVG_SITE_KMEANS_DRAIN,
 };
 
 __device__ __forceinline__ void record_error(uint32_t status, uint32_t site) {
@@ -149,35 +150,6 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
-}
-
-// 2^x for two values on the FMA pipe (no MUFU), x <= 8: Cody-Waite style
-// range reduction 2^x = 2^j * 2^f with j = round(x) (taken from the low
-// mantissa bits of x + 1.5 * 2^23) and f = x - j in [-1/2, 1/2], then a
-// degree-3 polynomial fitted here to 2^f on [-1/2, 1/2] by weighted least
-// squares (relative error below 7.5e-5, under the 2^-9 rounding of the bf16
-// probabilities it feeds).  2^j is applied by adding j to the exponent field.
-// Arguments below -125 (masked scores are -inf) are clamped to -125, whose
-// 2^x (about 2.4e-38) is negligible in a probability row.
-__device__ __forceinline__ float2 exp2_poly_x2(float2 x) {
-  constexpr float kMagic = 12582912.f;   // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 y = add_f32x2(x, make_float2(kMagic, kMagic));            // low bits of y hold round(x)
-  const float2 j = add_f32x2(y, make_float2(-kMagic, -kMagic));
-  const float2 f = fma_f32x2(j, make_float2(-1.f, -1.f), x);
-  float2 pl = fma_f32x2(f, make_float2(0.055171624f, 0.055171624f), make_float2(0.24261113f, 0.24261113f));
-  pl = fma_f32x2(pl, f, make_float2(0.69326097f, 0.69326097f));
-  pl = fma_f32x2(pl, f, make_float2(0.99992806f, 0.99992806f));
-  // 1.5 * 2^23 has nine zero low bits, so bits(y) << 23 is exactly j << 23
-  return make_float2(__int_as_float(__float_as_int(pl.x) + (__float_as_int(y.x) << 23)),
-                     __int_as_float(__float_as_int(pl.y) + (__float_as_int(y.y) << 23)));
-}
-
-// Two positive floats rounded to bf16 (half-up on the dropped 16 bits) and
-// packed low/high, with integer ops instead of a conversion instruction.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 // Maximum of three floats in one instruction.
@@ -525,26 +497,6 @@ __device__ __forceinline__ void mma_chain(uint32_t d_tmem, SmemDesc a, SmemDesc 
     const uint32_t ao = ((k >> 2) * A_HALF + (k & 3) * A_K) >> 4;
     const uint32_t bo = ((k >> 2) * B_HALF + (k & 3) * B_K) >> 4;
     mma_bf16_ss_off(d_tmem, a, ao, b, bo, idesc, k > 0 ? 1u : accumulate_first);
-  }
-}
-
-// A chain of STEPS K16 MMAs into one accumulator with A in tensor memory
-// (K-major: two bf16 per 32-bit column, 8 columns per K-step) and B in
-// shared memory, K-step k of B at byte offset (k / 4) * B_HALF + (k % 4) * B_K.
-template <int STEPS, uint32_t B_HALF, uint32_t B_K>
-__device__ __forceinline__ void mma_chain_ts(uint32_t d_tmem, uint32_t a_tmem, SmemDesc b,
-                                             uint32_t idesc, uint32_t accumulate_first) {
-#pragma unroll
-  for (int k = 0; k < STEPS; ++k) {
-    const uint32_t bo = ((k >> 2) * B_HALF + (k & 3) * B_K) >> 4;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
-        "mov.b64 bd, {%2, %3};\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem + 8 * k), "r"(b.lo + bo), "r"(b.hi), "r"(idesc),
-        "r"(k > 0 ? 1u : accumulate_first)
-        : "memory");
   }
 }
 

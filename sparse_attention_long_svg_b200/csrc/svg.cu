@@ -136,9 +136,14 @@ KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
   return w;
 }
 
+// The attention kernel runs at most this many CTAs (one per SM); each has
+// two slots of merged key ranges in the workspace (one per item in flight).
+constexpr int kAttnMaxCtas = 160;
+
 struct AttnWs {
   int32_t *num_items, *next_item, *qtiles, *ktiles;
   AttnItem *items;
+  int2 *ranges;
 };
 AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
   Carve c{static_cast<uint8_t *>(ws)};
@@ -148,6 +153,7 @@ AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
   w.qtiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.ktiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + kItemRows - 1) / kItemRows + Cq));
+  w.ranges = c.take<int2>(static_cast<size_t>(kAttnMaxCtas) * 2 * AttnCfg<128>::MAX_SEL);
   *bytes = c.used;
   return w;
 }
@@ -313,15 +319,21 @@ void svg_set_wait_timeout_ns(uint64_t ns) { g_wait_ns = ns ? ns : kDefaultWaitNs
 
 void svg_debug_set_fault(int fault) { g_fault = fault; }
 
-svg_status svg_get_error(svg_stream_t stream) {
+svg_status svg_get_error_detail(svg_stream_t stream, int32_t *site, int32_t *block) {
+  if (site) *site = 0;
+  if (block) *block = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return SVG_ERR_CUDA;
   uint32_t word = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return SVG_ERR_CUDA;
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return SVG_ERR_CUDA;
+  if (site) *site = static_cast<int32_t>((word >> 8) & 0xFFu);
+  if (block) *block = static_cast<int32_t>(word >> 16);
   return static_cast<svg_status>(word & 0xFFu);
 }
+
+svg_status svg_get_error(svg_stream_t stream) { return svg_get_error_detail(stream, nullptr, nullptr); }
 
 // ------------------------------------------------------------------ k-means
 size_t svg_kmeans_workspace_size(int BH, int N, int D, int C) {
@@ -549,6 +561,7 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   prm.op = static_cast<__nv_bfloat16 *>(op);
   prm.lse = lse;
   prm.perm = perm;
+  prm.ranges = w.ranges;
   prm.issued = nullptr;
   if (g_prof.on) {
     prm.issued = static_cast<unsigned long long *>(issued_pairs_address());
@@ -561,7 +574,7 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.wait_ns = g_wait_ns;
   prm.fault = g_fault;
-  const int grid = num_sms();
+  const int grid = num_sms() < kAttnMaxCtas ? num_sms() : kAttnMaxCtas;
   cudaEvent_t *pe = prof_slot(1);
   if (pe) cudaEventRecord(pe[0], s);
   if (D == 128) {
