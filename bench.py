@@ -313,15 +313,22 @@ def run_svg(args, wl):
         if ev:
             ev[2].record()
         svg.permute(layer.assign_q, wl.cq, [q], [layer.qp], layer.perm_q, layer.q_off, layer.workspace)
-        svg.permute(layer.assign_k, wl.ck, [k, v], [layer.kp, layer.vp], layer.perm_k, layer.k_off,
-                    layer.workspace)
+        if args.kv_gather:       # K permutation only: attention fetches K/V rows through it
+            svg.permute(layer.assign_k, wl.ck, [], [], layer.perm_k, layer.k_off, layer.workspace)
+        else:
+            svg.permute(layer.assign_k, wl.ck, [k, v], [layer.kp, layer.vp], layer.perm_k, layer.k_off,
+                        layer.workspace)
         if ev:
             ev[3].record()
         svg.select_topp(mu_q, layer.n_q, mu_k, layer.n_k, p, 0.0, layer.sel_count, layer.sel_cols)
         if ev:
             ev[4].record()
-        svg.sparse_attn(layer.qp, layer.kp, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
-                        layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
+        if args.kv_gather:
+            svg.sparse_attn_gather(layer.qp, k, v, layer.perm_k, layer.q_off, layer.k_off, layer.sel_count,
+                                   layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
+        else:
+            svg.sparse_attn(layer.qp, layer.kp, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
+                            layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
         if ev:
             ev[5].record()
 
@@ -392,7 +399,7 @@ def run_svg(args, wl):
         dv.copy_(hv, non_blocking=True)
         mu_q.copy_(hmq, non_blocking=True)
         mu_k.copy_(hmk, non_blocking=True)
-        o, _ = layer(dq, dk, dv, mu_q, mu_k, T, p, 0.0, out)
+        o, _ = layer(dq, dk, dv, mu_q, mu_k, T, p, 0.0, out, kv_gather=bool(args.kv_gather))
         hout.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
@@ -472,7 +479,9 @@ def run_svg(args, wl):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl, world, BH, T, p),
+            "config": dict(workload_config(wl, world, BH, T, p),
+                           kv=("gathered by the attention kernel through the K permutation" if args.kv_gather
+                               else "permuted copies written by svg_permute")),
             "attn_ms": stage_ms["attn+unpermute"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
             "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
@@ -512,6 +521,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="svg", choices=["svg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--top-p", type=float, default=None, help="override the workload's (first) top-p")
+    ap.add_argument("--kv-gather", type=int, default=0, choices=[0, 1],
+                    help="1: no permuted K/V copies; the attention kernel gathers K/V rows through the K permutation")
     ap.add_argument("--heads", type=int, default=None,
                     help="first H heads of the workload only (smaller case for profiler captures)")
     args = ap.parse_args(argv)

@@ -183,6 +183,32 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
                                       void *o, float *lse, void *ws, size_t ws_bytes,
                                       svg_stream_t stream);
 
+/* Attention with K and V in token order (section 2(c) "Customized attention
+ * kernel": the selected key rows are loaded sparsely from where they are and
+ * computed on densely): the kernel fetches permuted key row r of head h from
+ * row perm_k[h][r] of k and v with 16-byte asynchronous copies, so no
+ * permuted copy of K or V exists.  Q is permuted (dense query tiles).
+ *
+ *   qp      [BH, N, D] bf16   Q permuted by the Q permutation
+ *   k, v    [BH, N, D] bf16   K and V in token order
+ *   perm_k  [BH, N]    int32  the K permutation (svg_permute of the K
+ *                             clusters with ntensors = 0): perm_k[h][r] = token
+ *                             of permuted key row r; k_off its offsets
+ *   perm_q  [BH, N]    int32  optional: with it o (and lse) are stored in
+ *                             token order as in svg_sparse_attn_unpermuted;
+ *                             NULL stores Q-permuted rows as svg_sparse_attn
+ *   o       [BH, N, D] bf16   out; must not alias k or v (nor qp with perm_q)
+ * The other arguments, the workspace and the result are those of
+ * svg_sparse_attn (with perm_q: svg_sparse_attn_unpermuted).  A perm_k entry
+ * outside [0, N) is replaced by 0 and flagged with SVG_ERR_DEVICE_CHECK.
+ */
+svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, const int32_t *perm_k,
+                                  int BH, int N, int D, const int32_t *q_off, int Cq,
+                                  const int32_t *k_off, int Ck, const int32_t *sel_count,
+                                  const int32_t *sel_cols, float scale, const int32_t *perm_q,
+                                  void *o, float *lse, void *ws, size_t ws_bytes,
+                                  svg_stream_t stream);
+
 /* ------------------------------------------------------------------------ sparse attention, no allocation
  * No counterpart on the pages: this is a service for callers that cannot hand
  * the library a scratch buffer.  Some callers have no way to obtain device

@@ -48,6 +48,8 @@ SIGNATURES = {
     "svg_sparse_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _SZ, _P]),
     "svg_sparse_attn_unpermuted": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
                                         _SZ, _P]),
+    "svg_sparse_attn_gather": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
+                                    _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "svg_sparse_attn_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P]),
     "svg_profile_enable": (_I, [_I]),
@@ -274,6 +276,35 @@ def sparse_attn(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.
     return op, lse
 
 
+def sparse_attn_gather(qp, k, v, perm_k, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
+                       want_lse: bool = False, lse=None, workspace=None, stream=None, perm_q=None):
+    """Attention over the selected blocks with K and V in token order: the kernel
+    fetches key rows through ``perm_k`` (the K permutation), so no permuted K/V
+    copy exists.  Q is permuted.  With ``perm_q`` the output (and lse) come back
+    in token order, else in the Q-permuted order.  Returns (op, lse or None).
+    """
+    lib = load_library()
+    for t, n in ((qp, "qp"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(perm_k, "perm_k", torch.int32, 2)
+    BH, N, D = qp.shape
+    Cq = q_off.shape[1] - 1
+    Ck = k_off.shape[1] - 1
+    if op is None:
+        op = torch.empty_like(qp)
+    if want_lse and lse is None:
+        lse = torch.empty((BH, N), dtype=torch.float32, device=qp.device)
+    if workspace is None:
+        workspace = _ws(lib.svg_sparse_attn_workspace_size(BH, N, Cq), qp.device)
+    if perm_q is not None:
+        _need(perm_q, "perm_q", torch.int32, 2)
+    _check("svg_sparse_attn_gather", lib.svg_sparse_attn_gather(
+        _ptr(qp), _ptr(k), _ptr(v), _ptr(perm_k), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck, _ptr(sel_count),
+        _ptr(sel_cols), float(scale), _ptr(perm_q), _ptr(op), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return op, lse
+
+
 def sparse_attn_noalloc(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
                        want_lse: bool = False, lse=None, stream=None):
     """sparse_attn for callers that cannot provide device scratch memory.
@@ -327,8 +358,8 @@ class LayerState:
     sel_count: torch.Tensor
     sel_cols: torch.Tensor
     qp: torch.Tensor
-    kp: torch.Tensor
-    vp: torch.Tensor
+    kp: Optional[torch.Tensor]     # permuted K and V; None when attention gathered rows through perm_k
+    vp: Optional[torch.Tensor]
     op: Optional[torch.Tensor]     # permuted output; None when the un-permutation was fused
 
 
@@ -360,15 +391,31 @@ class SvgLayer:
         self.workspace = _ws(ws, device)
 
     def __call__(self, q, k, v, mu_q, mu_k, iters: int, p: float, scale: float = 0.0, out=None, stream=None,
-                 fused_unpermute: bool = True):
+                 fused_unpermute: bool = True, kv_gather: bool = False):
         """One layer; with ``fused_unpermute`` the attention kernel stores rows in token order
-        (no permuted output copy, ``LayerState.op`` is None), else attention + svg_unpermute."""
+        (no permuted output copy, ``LayerState.op`` is None), else attention + svg_unpermute.
+        With ``kv_gather`` K and V are not permuted: the attention kernel fetches their rows
+        through the K permutation (``LayerState.kp``/``vp`` are None); requires fused_unpermute."""
         kmeans(q, mu_q, iters, self.assign_q, self.n_q, self.workspace, stream)
         kmeans(k, mu_k, iters, self.assign_k, self.n_k, self.workspace, stream)
         Cq, Ck = mu_q.shape[1], mu_k.shape[1]
         permute(self.assign_q, Cq, [q], [self.qp], self.perm_q, self.q_off, self.workspace, stream)
-        permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace, stream)
+        if kv_gather:
+            if not fused_unpermute:
+                raise ValueError("kv_gather requires fused_unpermute")
+            permute(self.assign_k, Ck, [], [], self.perm_k, self.k_off, self.workspace, stream)
+        else:
+            permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace, stream)
         select_topp(mu_q, self.n_q, mu_k, self.n_k, p, scale, self.sel_count, self.sel_cols, stream)
+        if kv_gather:
+            if out is None:
+                out = torch.empty_like(q)
+            sparse_attn_gather(self.qp, k, v, self.perm_k, self.q_off, self.k_off, self.sel_count,
+                               self.sel_cols, scale, out, workspace=self.workspace, stream=stream,
+                               perm_q=self.perm_q)
+            return out, LayerState(mu_q, mu_k, self.assign_q, self.assign_k, self.n_q, self.n_k, self.perm_q,
+                                   self.perm_k, self.q_off, self.k_off, self.sel_count, self.sel_cols, self.qp,
+                                   None, None, None)
         if fused_unpermute:
             if out is None:
                 out = torch.empty_like(q)

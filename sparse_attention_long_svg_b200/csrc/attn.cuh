@@ -65,6 +65,7 @@ constexpr int kItemReaders = 11;
 template <int D>
 struct AttnCfg {
   static constexpr int BM = 128, BN = 128, SLOT = 8, NSLOT = BN / SLOT;
+  static constexpr int HEAD_DIM = D;
   static constexpr int DH = D / 64;                   // 64-channel (128-byte) halves
   static constexpr int KST = D == 128 ? 2 : 4;        // K ring slots (same for V)
   static constexpr int QT_BYTES = BM * D * 2;         // one Q tile
@@ -95,6 +96,9 @@ struct AttnCfg {
 // TMA boxes of 8, 16, 32, 64 and 128 rows (one tensor map each for K and V).
 constexpr int kNumBoxSizes = 5;
 
+// Box mode (K and V already permuted): k[b], v[b] have boxes of 8 << b rows.
+// Gather mode (K and V in token order, rows fetched through the K
+// permutation with 16-byte asynchronous copies): k and v are unused.
 struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k[kNumBoxSizes];
@@ -140,6 +144,8 @@ struct AttnParams {
   __nv_bfloat16 *op;
   float *lse;
   const int32_t *perm;   // optional: write row r of a head to row perm[r] (un-permuted output)
+  const int32_t *perm_k; // gather mode: permuted key row r of a head is row perm_k[r] of K and V
+  const __nv_bfloat16 *kg, *vg;   // gather mode: K and V [BH, N, D] in token order
   unsigned long long *issued;   // optional: += (query tile, key tile) pairs issued
   int2 *ranges;          // per CTA: 2 x MAX_SEL merged key runs (first row, rows), one slot per header slot
   int N, Cq, Ck, BH;
@@ -211,7 +217,42 @@ __device__ __forceinline__ int attn_sel_count(const int32_t *sel_count, size_t r
   return c;
 }
 
-template <int D>
+// Gather mode: one 128-row key tile (K or V) into a ring slot, in the same
+// 128-byte-swizzled K-major layout the tensor-map loads produce (row r,
+// 16-byte chunk c of 64-channel half h at h * HALF_KV + 128 r + 16 (c ^ r % 8)).
+// Lane l holds the global rows of tile rows 4 l .. 4 l + 3 in `rows`; each
+// warp instruction copies D / 8 consecutive 16-byte chunks of 32 / (D / 8)
+// rows (coalesced), the rows taken from their owners by shuffles.
+template <class Cfg>
+__device__ __forceinline__ void gather_rows(uint32_t slot_addr, const __nv_bfloat16 *__restrict__ src, int4 rows,
+                                            int lane) {
+  constexpr int LPR = Cfg::HEAD_DIM / 8;   // lanes (16-byte chunks) per row
+  constexpr int RPI = 32 / LPR;        // rows per instruction
+  const int sub = lane / LPR, c = lane % LPR;
+  const uint32_t half_off = static_cast<uint32_t>((c >> 3) * Cfg::HALF_KV);
+  const int cc = c & 7;
+#pragma unroll
+  for (int i = 0; i < Cfg::BN / RPI; ++i) {
+    const int r0 = i * RPI;            // tile rows r0 .. r0 + RPI - 1 (one owner lane per 4 rows)
+    int v[RPI];
+#pragma unroll
+    for (int k = 0; k < RPI; ++k) {
+      const int r = r0 + k;
+      const int comp = r & 3;
+      v[k] = __shfl_sync(0xffffffffu, comp == 0 ? rows.x : comp == 1 ? rows.y : comp == 2 ? rows.z : rows.w, r >> 2);
+    }
+    int g = v[0];
+#pragma unroll
+    for (int k = 1; k < RPI; ++k)
+      if (sub == k) g = v[k];
+    const int r = r0 + sub;
+    const uint32_t dst = slot_addr + half_off + static_cast<uint32_t>(r * 128) +
+                         (static_cast<uint32_t>(cc ^ (r & 7)) << 4);
+    cp_async_16(dst, src + static_cast<size_t>(g) * Cfg::HEAD_DIM + c * 8);
+  }
+}
+
+template <int D, bool GATHER>
 __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams P) {
   using Cfg = AttnCfg<D>;
@@ -229,8 +270,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
-      mbar_init(&B->k_full[s], 1);
-      mbar_init(&B->v_full[s], 1);
+      mbar_init(&B->k_full[s], GATHER ? 32 : 1);   // gather mode: one arrival per producer lane
+      mbar_init(&B->v_full[s], GATHER ? 32 : 1);
       for (int x = 0; x < 2; ++x) {
         mbar_init(&B->k_empty[x][s], 1);
         mbar_init(&B->v_empty[x][s], 1);
@@ -260,7 +301,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   }
   if (warp == Cfg::PRODUCER_WARP && lane == 0) {
     tma_prefetch_desc(&maps.q);
-    for (int b = 0; b < kNumBoxSizes; ++b) {
+    for (int b = 0; b < (GATHER ? 0 : kNumBoxSizes); ++b) {
       tma_prefetch_desc(&maps.k[b]);
       tma_prefetch_desc(&maps.v[b]);
     }
@@ -382,9 +423,18 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       // the tile-B releases of that slot expected so far
       uint32_t slot_b = 0, rel_b = 0, nq_b = 0;
       uint32_t tile_b = 0;               // bit e: box-ring entry e has tile B
-      int box_row[kBoxRing], box_code[kBoxRing];   // this lane's box of each entry: row, kind | slot << 8 (-1: none)
+      // box mode: this lane's box of each entry (row, kind | slot << 8; -1: none);
+      // gather mode: this lane's four key rows of each entry (rows 4 lane .. +3 of the tile)
+      int box_row[kBoxRing], box_code[kBoxRing];
+      int4 grow[GATHER ? kBoxRing : 1];
 #pragma unroll
       for (int e = 0; e < kBoxRing; ++e) box_row[e] = box_code[e] = -1;
+#pragma unroll
+      for (int e = 0; e < (GATHER ? kBoxRing : 1); ++e) grow[e] = make_int4(0, 0, 0, 0);
+      const int32_t *perm_k = P.perm_k;
+      bool pre = false;                  // gather mode: the next key tile's rows are looked up
+      uint32_t pre_mask[4] = {0, 0, 0, 0};
+      int4 pre_src = make_int4(0, 0, 0, 0);
       uint32_t gk = 0, gv = 0, nq = 0, nq1 = 0;   // K and V tiles issued, Q loads issued (all, tile B)
       int n = 0;                         // next item (header slot n & 1)
       bool k_active = false, k_done = false, prev_b = false;
@@ -434,21 +484,14 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           }
         }
         // ---- K side: the next key tile of the item
-        if (k_active && gk - gv < static_cast<uint32_t>(kBoxRing)) {
-          const int slot = static_cast<int>(gk % Cfg::KST);
-          const uint32_t sbit = 1u << slot;
-          const bool free_slot =
-              gk < static_cast<uint32_t>(Cfg::KST) ||
-              (test(&B->k_empty[0][slot], ((gk / Cfg::KST) - 1) & 1) &&
-               (!(slot_b & sbit) || test(&B->k_empty[1][slot], (rel_b & sbit) ? 0u : 1u)));
-          if (free_slot) {
-            // cut the tile into boxes of 1..16 slots (8..128 rows): the largest
-            // power of two that fits both the tile and the rest of the run
-            const int rb = static_cast<int>(gk % kBoxRing);
-            const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
-            uint32_t mask[4] = {0, 0, 0, 0};
-            int sl = 0, nb = 0, my_row = -1, my_code = -1;
-            while (sl < Cfg::NSLOT) {
+        if constexpr (GATHER) {
+          // gather mode: the next key tile's rows are looked up (the loads of
+          // its K-permutation entries issued) as soon as it may be built, so
+          // they are in registers by the time its slot frees
+          if (k_active && !pre && gk - gv < static_cast<uint32_t>(kBoxRing)) {
+            pre_mask[0] = pre_mask[1] = pre_mask[2] = pre_mask[3] = 0;
+            int my_p0 = 0, my_nv = 0;    // first permuted row and valid rows of this lane's slot
+            for (int sl = 0; sl < Cfg::NSLOT; ++sl) {
               while (left <= 0 && ci < cnt) {
                 if ((ci & ~31) != win_base) {   // refill the window: ranges [ci & ~31, +32)
                   win_base = ci & ~31;
@@ -458,47 +501,121 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                 left = __shfl_sync(0xffffffffu, win.y, ci & 31);
                 ++ci;
               }
-              const int space = Cfg::NSLOT - sl;
-              const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
-              int kind = 0;
-              while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
-              const int nsl = 1 << kind;
-              if (lane == nb) {
-                my_row = left > 0 ? it.h * P.N + cur : pad_row;
-                my_code = kind | (sl << 8);
+              const int nv = left > 0 ? min(left, Cfg::SLOT) : 0;
+              if ((lane >> 1) == sl) {   // padding slots re-read row 0; they are masked
+                my_p0 = nv > 0 ? cur : 0;
+                my_nv = nv;
               }
-              if (left > 0) {
-                set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
-                cur += nsl * Cfg::SLOT;
-                left -= nsl * Cfg::SLOT;
-              }
-              ++nb;
-              sl += nsl;
-            }
-#pragma unroll
-            for (int e = 0; e < kBoxRing; ++e) {
-              if (e == rb) {
-                box_row[e] = my_row;
-                box_code[e] = my_code;
+              if (nv > 0) {
+                set_bits(pre_mask, sl * Cfg::SLOT, nv);
+                cur += Cfg::SLOT;
+                left -= Cfg::SLOT;
               }
             }
-            tile_b = has_b ? (tile_b | (1u << rb)) : (tile_b & ~(1u << rb));
-            const int mi = static_cast<int>(gk % kMetaRing);
-            slot_b = has_b ? (slot_b | sbit) : (slot_b & ~sbit);
-            if (has_b) rel_b ^= sbit;
-            if (lane == 0) {
+            const int32_t *pk = perm_k + static_cast<size_t>(it.h) * P.N;
+            const int o = 4 * (lane & 1);
+            pre_src.x = __ldg(pk + my_p0 + (o < my_nv ? o : 0));
+            pre_src.y = __ldg(pk + my_p0 + (o + 1 < my_nv ? o + 1 : 0));
+            pre_src.z = __ldg(pk + my_p0 + (o + 2 < my_nv ? o + 2 : 0));
+            pre_src.w = __ldg(pk + my_p0 + (o + 3 < my_nv ? o + 3 : 0));
+            pre = true;
+          }
+        }
+        if (k_active && (!GATHER || pre) && gk - gv < static_cast<uint32_t>(kBoxRing)) {
+          const int slot = static_cast<int>(gk % Cfg::KST);
+          const uint32_t sbit = 1u << slot;
+          const bool free_slot =
+              gk < static_cast<uint32_t>(Cfg::KST) ||
+              (test(&B->k_empty[0][slot], ((gk / Cfg::KST) - 1) & 1) &&
+               (!(slot_b & sbit) || test(&B->k_empty[1][slot], (rel_b & sbit) ? 0u : 1u)));
+          if (free_slot) {
+            if constexpr (GATHER) {
+              const int rb = static_cast<int>(gk % kBoxRing);
+              const int src[4] = {pre_src.x, pre_src.y, pre_src.z, pre_src.w};
+              int rr[4];
+              bool bad = false;
 #pragma unroll
-              for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
-              mbar_arrive(&B->meta_full[mi]);
-              mbar_arrive_expect_tx(&B->k_full[slot], Cfg::KV_BYTES);
-            }
-            __syncwarp();
-            if (my_code >= 0) {
-              const int kind = my_code & 0xFF, at = my_code >> 8;
+              for (int i = 0; i < 4; ++i) {
+                const bool out = src[i] < 0 || src[i] >= P.N;
+                bad |= out;
+                rr[i] = it.h * P.N + (out ? 0 : src[i]);
+              }
+              if (bad) record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_PRODUCER);
+              pre = false;
+              const int4 r4 = make_int4(rr[0], rr[1], rr[2], rr[3]);
 #pragma unroll
-              for (int dh = 0; dh < Cfg::DH; ++dh)
-                tma_load_2d(sK + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64,
-                            my_row, &B->k_full[slot]);
+              for (int e = 0; e < kBoxRing; ++e)
+                if (e == rb) grow[e] = r4;
+              tile_b = has_b ? (tile_b | (1u << rb)) : (tile_b & ~(1u << rb));
+              const int mi = static_cast<int>(gk % kMetaRing);
+              slot_b = has_b ? (slot_b | sbit) : (slot_b & ~sbit);
+              if (has_b) rel_b ^= sbit;
+              if (lane == 0) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) B->meta[mi][w] = pre_mask[w];
+                mbar_arrive(&B->meta_full[mi]);
+              }
+              gather_rows<Cfg>(smem_u32(sK + slot * Cfg::KV_BYTES), P.kg, r4, lane);
+              cp_async_arrive(&B->k_full[slot]);
+            } else {
+              // cut the tile into boxes of 1..16 slots (8..128 rows): the largest
+              // power of two that fits both the tile and the rest of the run
+              const int rb = static_cast<int>(gk % kBoxRing);
+              const int pad_row = it.h * P.N;  // unused slots re-read a valid row; they are masked
+              uint32_t mask[4] = {0, 0, 0, 0};
+              int sl = 0, nb = 0, my_row = -1, my_code = -1;
+              while (sl < Cfg::NSLOT) {
+                while (left <= 0 && ci < cnt) {
+                  if ((ci & ~31) != win_base) {   // refill the window: ranges [ci & ~31, +32)
+                    win_base = ci & ~31;
+                    win = win_base + lane < cnt ? __ldcg(rng + win_base + lane) : make_int2(0, 0);
+                  }
+                  cur = __shfl_sync(0xffffffffu, win.x, ci & 31);
+                  left = __shfl_sync(0xffffffffu, win.y, ci & 31);
+                  ++ci;
+                }
+                const int space = Cfg::NSLOT - sl;
+                const int need = left > 0 ? (left + Cfg::SLOT - 1) / Cfg::SLOT : space;
+                int kind = 0;
+                while (kind + 1 < kNumBoxSizes && (2 << kind) <= space && (2 << kind) <= need) ++kind;
+                const int nsl = 1 << kind;
+                if (lane == nb) {
+                  my_row = left > 0 ? it.h * P.N + cur : pad_row;
+                  my_code = kind | (sl << 8);
+                }
+                if (left > 0) {
+                  set_bits(mask, sl * Cfg::SLOT, min(left, nsl * Cfg::SLOT));
+                  cur += nsl * Cfg::SLOT;
+                  left -= nsl * Cfg::SLOT;
+                }
+                ++nb;
+                sl += nsl;
+              }
+  #pragma unroll
+              for (int e = 0; e < kBoxRing; ++e) {
+                if (e == rb) {
+                  box_row[e] = my_row;
+                  box_code[e] = my_code;
+                }
+              }
+              tile_b = has_b ? (tile_b | (1u << rb)) : (tile_b & ~(1u << rb));
+              const int mi = static_cast<int>(gk % kMetaRing);
+              slot_b = has_b ? (slot_b | sbit) : (slot_b & ~sbit);
+              if (has_b) rel_b ^= sbit;
+              if (lane == 0) {
+  #pragma unroll
+                for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
+                mbar_arrive(&B->meta_full[mi]);
+                mbar_arrive_expect_tx(&B->k_full[slot], Cfg::KV_BYTES);
+              }
+              __syncwarp();
+              if (my_code >= 0) {
+                const int kind = my_code & 0xFF, at = my_code >> 8;
+  #pragma unroll
+                for (int dh = 0; dh < Cfg::DH; ++dh)
+                  tma_load_2d(sK + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64,
+                              my_row, &B->k_full[slot]);
+              }
             }
             ++gk;
             progress = true;
@@ -524,22 +641,31 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             const bool tb = (tile_b >> rb) & 1u;
             slot_b = tb ? (slot_b | sbit) : (slot_b & ~sbit);
             if (tb) rel_b ^= sbit;
-            int my_row = -1, my_code = -1;
+            if constexpr (GATHER) {
+              int4 r4 = grow[0];
 #pragma unroll
-            for (int e = 0; e < kBoxRing; ++e) {
-              if (e == rb) {
-                my_row = box_row[e];
-                my_code = box_code[e];
+              for (int e = 1; e < kBoxRing; ++e)
+                if (e == rb) r4 = grow[e];
+              gather_rows<Cfg>(smem_u32(sV + slot * Cfg::KV_BYTES), P.vg, r4, lane);
+              cp_async_arrive(&B->v_full[slot]);
+            } else {
+              int my_row = -1, my_code = -1;
+  #pragma unroll
+              for (int e = 0; e < kBoxRing; ++e) {
+                if (e == rb) {
+                  my_row = box_row[e];
+                  my_code = box_code[e];
+                }
               }
-            }
-            if (lane == 0) mbar_arrive_expect_tx(&B->v_full[slot], Cfg::KV_BYTES);
-            __syncwarp();
-            if (my_code >= 0) {
-              const int kind = my_code & 0xFF, at = my_code >> 8;
-#pragma unroll
-              for (int dh = 0; dh < Cfg::DH; ++dh)
-                tma_load_2d(sV + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64,
-                            my_row, &B->v_full[slot]);
+              if (lane == 0) mbar_arrive_expect_tx(&B->v_full[slot], Cfg::KV_BYTES);
+              __syncwarp();
+              if (my_code >= 0) {
+                const int kind = my_code & 0xFF, at = my_code >> 8;
+  #pragma unroll
+                for (int dh = 0; dh < Cfg::DH; ++dh)
+                  tma_load_2d(sV + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64,
+                              my_row, &B->v_full[slot]);
+              }
             }
             ++gv;
             progress = true;
@@ -619,6 +745,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               ok = false;
               break;
             }
+            if constexpr (GATHER) fence_proxy_async_smem();   // cp.async writes -> tensor-core reads
             tc_fence_after();
             mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
                 tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
@@ -632,6 +759,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
               ok = false;
               break;
             }
+            if constexpr (GATHER) fence_proxy_async_smem();
             tc_fence_after();
             // A = P [128 q x 128 keys], K-major in two 64-key halves; B = V [128 keys x D],
             // MN-major, 16 keys = 2048 bytes per K-step

@@ -514,13 +514,14 @@ size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq) {
 namespace {
 // Shared body of svg_sparse_attn (perm == nullptr: permuted output rows) and
 // svg_sparse_attn_unpermuted (row r of a head stored at row perm[r]).
-svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int BH, int N, int D,
-                            const int32_t *q_off, int Cq, const int32_t *k_off, int Ck,
-                            const int32_t *sel_count, const int32_t *sel_cols, float scale,
+svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, const int32_t *perm_k,
+                            int BH, int N, int D, const int32_t *q_off, int Cq, const int32_t *k_off,
+                            int Ck, const int32_t *sel_count, const int32_t *sel_cols, float scale,
                             const int32_t *perm, void *op, float *lse, void *ws, size_t ws_bytes,
                             svg_stream_t stream) {
   if (!qp || !kp || !vp || !q_off || !k_off || !sel_count || !sel_cols || !op || !ws)
     return SVG_ERR_INVALID_ARG;
+  const bool gather = perm_k != nullptr;
   if (perm != nullptr && (op == qp || op == kp || op == vp)) return SVG_ERR_INVALID_ARG;
   if (!sizes_ok(BH, N) || Cq < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
@@ -544,11 +545,11 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   if (st != SVG_OK) return st;
 
   AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
   const uint64_t rows = static_cast<uint64_t>(BH) * N;
   if (!make_map_bf16(&maps.q, qp, rows, D, 128)) return SVG_ERR_CUDA;
-  for (int b = 0; b < kNumBoxSizes; ++b)
-    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b) ||
-        !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
+  for (int b = 0; b < (gather ? 0 : kNumBoxSizes); ++b)   // gather mode copies rows without tensor maps
+    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b) || !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
       return SVG_ERR_CUDA;
   AttnParams prm;
   prm.q_off = q_off;
@@ -561,6 +562,9 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   prm.op = static_cast<__nv_bfloat16 *>(op);
   prm.lse = lse;
   prm.perm = perm;
+  prm.perm_k = perm_k;
+  prm.kg = static_cast<const __nv_bfloat16 *>(kp);
+  prm.vg = static_cast<const __nv_bfloat16 *>(vp);
   prm.ranges = w.ranges;
   prm.issued = nullptr;
   if (g_prof.on) {
@@ -577,15 +581,19 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, int 
   const int grid = num_sms() < kAttnMaxCtas ? num_sms() : kAttnMaxCtas;
   cudaEvent_t *pe = prof_slot(1);
   if (pe) cudaEventRecord(pe[0], s);
-  if (D == 128) {
-    using Cfg = AttnCfg<128>;
-    if (!set_smem(sparse_attn_kernel<128>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
-    sparse_attn_kernel<128><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
-  } else {
-    using Cfg = AttnCfg<64>;
-    if (!set_smem(sparse_attn_kernel<64>, Cfg::SMEM_BYTES)) return SVG_ERR_CUDA;
-    sparse_attn_kernel<64><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(maps, prm);
-  }
+  auto launch = [&](auto kernel, int threads, int smem) {
+    if (!set_smem(kernel, smem)) return false;
+    kernel<<<grid, threads, smem, s>>>(maps, prm);
+    return true;
+  };
+  bool ok;
+  if (D == 128)
+    ok = gather ? launch(sparse_attn_kernel<128, true>, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES)
+                : launch(sparse_attn_kernel<128, false>, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES);
+  else
+    ok = gather ? launch(sparse_attn_kernel<64, true>, AttnCfg<64>::THREADS, AttnCfg<64>::SMEM_BYTES)
+                : launch(sparse_attn_kernel<64, false>, AttnCfg<64>::THREADS, AttnCfg<64>::SMEM_BYTES);
+  if (!ok) return SVG_ERR_CUDA;
   if (pe) cudaEventRecord(pe[1], s);
   return launch_status("sparse_attn_kernel");
 }
@@ -598,8 +606,8 @@ svg_status svg_sparse_attn(const void *qp, const void *kp, const void *vp, int B
                            const int32_t *sel_count, const int32_t *sel_cols, float scale,
                            void *op, float *lse, void *ws, size_t ws_bytes,
                            svg_stream_t stream) {
-  return sparse_attn_impl(qp, kp, vp, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale,
-                          nullptr, op, lse, ws, ws_bytes, stream);
+  return sparse_attn_impl(qp, kp, vp, nullptr, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols,
+                          scale, nullptr, op, lse, ws, ws_bytes, stream);
 }
 
 svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void *vp, int BH,
@@ -609,8 +617,20 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
                                       void *o, float *lse, void *ws, size_t ws_bytes,
                                       svg_stream_t stream) {
   if (!perm_q) return SVG_ERR_INVALID_ARG;
-  return sparse_attn_impl(qp, kp, vp, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale,
-                          perm_q, o, lse, ws, ws_bytes, stream);
+  return sparse_attn_impl(qp, kp, vp, nullptr, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols,
+                          scale, perm_q, o, lse, ws, ws_bytes, stream);
+}
+
+svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, const int32_t *perm_k,
+                                  int BH, int N, int D, const int32_t *q_off, int Cq,
+                                  const int32_t *k_off, int Ck, const int32_t *sel_count,
+                                  const int32_t *sel_cols, float scale, const int32_t *perm_q,
+                                  void *o, float *lse, void *ws, size_t ws_bytes,
+                                  svg_stream_t stream) {
+  if (!perm_k) return SVG_ERR_INVALID_ARG;
+  if (o == k || o == v) return SVG_ERR_INVALID_ARG;
+  return sparse_attn_impl(qp, k, v, perm_k, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols,
+                          scale, perm_q, o, lse, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -237,6 +237,63 @@ def test_fused_unpermute_equals_separate_pass(name, case_data):
     assert torch.equal(lse_o, lse_want)
 
 
+def oracle_blocks(ref, Cq, Ck):
+    """The oracle's selection as (sel_count [H, Cq], sel_cols [H, Cq, Ck]) arrays."""
+    H = len(ref)
+    cnt = np.zeros((H, Cq), np.int32)
+    cols = np.full((H, Cq, Ck), -1, np.int32)
+    for h in range(H):
+        for i, s in enumerate(ref[h].selection):
+            cnt[h, i] = len(s.cols)
+            cols[h, i, :len(s.cols)] = s.cols
+    return cnt, cols
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_gather_kv_equals_permuted_kv(name, case_data):
+    """svg_sparse_attn_gather (K, V in token order, key rows fetched through perm_k) equals
+    svg_sparse_attn on permuted K, V bit for bit, with and without the fused
+    un-permutation (lse too); the latter is checked against the oracle above."""
+    L, ref = case_data(name)
+    qp, kp, vp, q_off, k_off, op, lse = run_attention_from_oracle(L, ref)
+    cnt, cols = oracle_blocks(ref, q_off.shape[1] - 1, k_off.shape[1] - 1)
+    perm_k = dev_i32(np.stack([r.perm_k for r in ref]))
+    perm_q = dev_i32(np.stack([r.perm_q for r in ref]))
+    args = (dev_i32(q_off), dev_i32(k_off), dev_i32(cnt), dev_i32(cols))
+    k, v = dev_bf16(L.k), dev_bf16(L.v)
+    og, lg = svg.sparse_attn_gather(dev_bf16(qp), k, v, perm_k, *args, want_lse=True)
+    torch.cuda.synchronize()
+    assert svg.get_error() == 0
+    assert torch.equal(og, op)
+    assert torch.equal(lg, lse)
+    ou, lu = svg.sparse_attn_gather(dev_bf16(qp), k, v, perm_k, *args, want_lse=True, perm_q=perm_q)
+    torch.cuda.synchronize()
+    assert svg.get_error() == 0
+    assert torch.equal(ou, svg.unpermute(op, perm_q))
+    lse_want = torch.empty_like(lse)
+    lse_want.scatter_(1, perm_q.long(), lse)
+    assert torch.equal(lu, lse_want)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_kv_gather_equals_permuted_layer(name, case_data):
+    """The layer with K/V gathered inside attention gives the same output, bit for bit."""
+    L, _ = case_data(name)
+    H, N, D = L.q.shape
+    wl = L.workload
+    outs = []
+    for gather in (False, True):
+        layer = svg.SvgLayer(H, N, D, wl.cq, wl.ck)
+        mu_q, mu_k = dev_f32(L.init_centroids("q")), dev_f32(L.init_centroids("k"))
+        out, st = layer(dev_bf16(L.q), dev_bf16(L.k), dev_bf16(L.v), mu_q, mu_k, wl.iters, top_p_of(wl),
+                        kv_gather=gather)
+        torch.cuda.synchronize()
+        assert svg.get_error() == 0
+        assert (st.kp is None) == gather
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])
+
+
 def test_sparse_attention_all_blocks_equals_dense(case_data):
     L, ref = case_data("tiny")
     H, N, D = L.q.shape
