@@ -28,28 +28,40 @@ def _lib():
     svg.load_library()
 
 
-def test_timeout_is_reported_and_context_stays_usable():
+ATTN_SITES = {"attention producer", "attention MMA issuer", "attention softmax", "attention drain"}
+
+
+@pytest.mark.parametrize("gather", [False, True], ids=["permuted-kv", "gathered-kv"])
+def test_timeout_is_reported_and_context_stays_usable(gather):
     lib = svg.load_library()
     wl = synth.small_workload("480p-5s", (5, 12, 20), heads=3, cq=6, ck=40, iters=3)
     L = synth.make_layer(wl)
     layer = svg.SvgLayer(*L.q.shape, wl.cq, wl.ck)
-    _, st = layer(dev_bf16(L.q), dev_bf16(L.k), dev_bf16(L.v), dev_f32(L.init_centroids("q")),
-                  dev_f32(L.init_centroids("k")), wl.iters, 0.9)
-    args = (st.qp, st.kp, st.vp, st.q_off, st.k_off, st.sel_count, st.sel_cols)
-    ref, _ = svg.sparse_attn(*args)
+    k, v = dev_bf16(L.k), dev_bf16(L.v)
+    _, st = layer(dev_bf16(L.q), k, v, dev_f32(L.init_centroids("q")), dev_f32(L.init_centroids("k")),
+                  wl.iters, 0.9)
+    blocks = (st.q_off, st.k_off, st.sel_count, st.sel_cols)
+
+    def attend():
+        if gather:
+            return svg.sparse_attn_gather(st.qp, k, v, st.perm_k, *blocks)
+        return svg.sparse_attn(st.qp, st.kp, st.vp, *blocks)
+    ref, _ = attend()
     ref = ref.clone()
     assert svg.get_error() == 0
     try:
         svg.set_wait_timeout_ns(20_000_000)          # 20 ms
         lib.svg_debug_set_fault(1)
-        svg.sparse_attn(*args)                       # the launch itself succeeds
-        status = svg.get_error()
+        attend()                                     # the launch itself succeeds
+        status, site, cta = svg.get_error_detail()
     finally:
         lib.svg_debug_set_fault(0)
         svg.set_wait_timeout_ns(0)                   # default bound
     assert status == 5, svg.STATUS.get(status, status)   # SVG_ERR_TIMEOUT
+    assert site in ATTN_SITES, site
+    assert 0 <= cta < 160
     assert svg.get_error() == 0                      # the word was cleared
-    again, _ = svg.sparse_attn(*args)
+    again, _ = attend()
     torch.cuda.synchronize()
     assert svg.get_error() == 0
     assert torch.equal(again, ref)
