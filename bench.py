@@ -496,6 +496,181 @@ def run_svg(args, wl):
     return 0
 
 
+# DynamicRad settings of the --mask dynrad-* legs (block of 256 tokens: two query
+# tiles per block; static density about 18 % and dynamic about 6 % on 480p-5s).
+DYNRAD = {"block": 256, "w0": 3.0, "gamma": 0.5, "rho0": 0.5, "theta": 1.0}
+
+
+def dynrad_oracle_sample(wl, heads: int, mode: str):
+    """The DynamicRad oracle (mask + attention) on the first `heads` heads: (seconds, attention FLOPs)."""
+    from oracle import dynrad_oracle as dr
+    L = synth.make_layer(wl, heads=heads)
+    H, N, D = L.q.shape
+    frames = wl.grid[0]
+    c = {k: float(np.float32(v)) for k, v in DYNRAD.items() if k != "block"}
+    t0 = time.perf_counter()
+    flops = 0.0
+    for h in range(H):
+        offs, nb = dr.block_layout(N, frames, DYNRAD["block"])
+        if mode == "static":
+            sel = dr.static_select(frames, nb, c["w0"], c["gamma"], c["rho0"])
+        else:
+            sel = [r.cols for r in dr.dynamic_select(L.q[h], L.k[h], offs, frames, nb, c["w0"], c["gamma"],
+                                                    c["theta"], 1.0 / math.sqrt(D))]
+        dr.attention(L.q[h], L.k[h], L.v[h], offs, sel, 1.0 / math.sqrt(D))
+        flops += 4.0 * D * dr.density(offs, sel)[0]
+    return time.perf_counter() - t0, flops
+
+
+def run_dynrad(args, wl):
+    """The DynamicRad workload on the same attention kernel: block masks (svg_dynrad_select) + attention
+    on Q, K, V in token order.  Same metric and timing rules as the SVG2 leg."""
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import sparse_attention_long_svg_b200 as svg
+    svg.load_library()
+    peaks, peak_kind = load_peaks()
+    mode = args.mask.split("-", 1)[1]
+    L = synth.make_layer(wl, heads=args.heads)
+    BH, N, D = L.q.shape
+    frames, B = wl.grid[0], DYNRAD["block"]
+
+    def to_dev(x):
+        return torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(device)
+    q, k, v = to_dev(L.q), to_dev(L.k), to_dev(L.v)
+    lib = svg.load_library()
+    Cb = lib.svg_dynrad_num_blocks(N, frames, B)
+    i32 = dict(dtype=torch.int32, device=device)
+    offs, cnt, cols = torch.empty((BH, Cb + 1), **i32), torch.empty((BH, Cb), **i32), torch.empty((BH, Cb, Cb), **i32)
+    ws = torch.empty(max(lib.svg_dynrad_workspace_size(BH, N, D, frames, B),
+                         lib.svg_sparse_attn_workspace_size(BH, N, Cb), 256), dtype=torch.uint8, device=device)
+    out = torch.empty_like(q)
+    prm = dict(w0=DYNRAD["w0"], gamma=DYNRAD["gamma"], rho0=DYNRAD["rho0"], theta=DYNRAD["theta"])
+
+    def step(qq, kk, vv, ev=None):
+        if ev:
+            ev[0].record()
+        svg.dynrad_select(qq, kk, frames, B, mode, offsets=offs, sel_count=cnt, sel_cols=cols, workspace=ws, **prm)
+        if ev:
+            ev[1].record()
+        svg.sparse_attn(qq, kk, vv, offs, offs, cnt, cols, 0.0, out, workspace=ws)
+        if ev:
+            ev[2].record()
+
+    clocks = ClockSampler(device.index)
+    clocks.__enter__()
+    for _ in range(args.warmup):
+        step(q, k, v)
+    torch.cuda.synchronize()
+    err = svg.get_error_detail()
+    if err[0] != 0:
+        raise RuntimeError("device error word set during warm-up: status %d at %s, CTA %d" % err)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    svg.profile_enable(True)
+    svg.profile_read("sparse_attn")
+    svg.profile_attn_pairs()
+    t_start.record()
+    for s in range(args.steps):
+        step(q, k, v, events[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
+    attn_k_ms, attn_n, _ = svg.profile_read("sparse_attn")
+    issued_pairs = svg.profile_attn_pairs()
+    svg.profile_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    local_ms = t_start.elapsed_time(t_end)
+    err = svg.get_error_detail()
+    if err[0] != 0:
+        raise RuntimeError("device error word set during the timed steps: status %d at %s, CTA %d" % err)
+    mask_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
+    o_h, c_h, s_h = offs.cpu().numpy(), cnt.cpu().numpy(), cols.cpu().numpy()
+    pairs = 0
+    for h in range(BH):
+        nb_sizes = np.diff(o_h[h])
+        for i in range(Cb):
+            pairs += int(nb_sizes[i]) * int(nb_sizes[s_h[h, i, :c_h[h, i]]].sum())
+    flops_layer = 4.0 * D * pairs
+    total_ms = reduce_max(local_ms, world, device)
+    value = reduce_sum(flops_layer * args.steps, world, device) / (total_ms * 1e-3) / 1e12
+
+    e2e_steps = max(1, min(args.steps, 10))
+    hq, hk, hv = (torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+                  for x in (L.q, L.k, L.v))
+    hout = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step(dq, dk, dv)
+        hout.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, device)
+    e2e_value = reduce_sum(flops_layer * e2e_steps, world, device) / (e2e_ms * 1e-3) / 1e12
+
+    tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tc_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    attn_kernel_ms = attn_k_ms / max(attn_n, 1)
+    attn_kernel_tflops = flops_layer / (attn_kernel_ms * 1e-3) / 1e12
+    issued = 4.0 * D * svg.ATTN_TILE * svg.ATTN_TILE * issued_pairs / max(attn_n, 1)
+    roofline = {"kernel": f"sparse_attn_kernel<{D}>", "bound": "tensor", "achieved": attn_kernel_tflops,
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_kernel_tflops / tc_peak,
+                "frac_of_sustained": attn_kernel_tflops / tc_sust, "traffic": None,
+                "peak_kind": f"{peak_kind} bf16 burst (each launch timed on its own)",
+                "launch_ms": attn_kernel_ms, "launches": attn_n,
+                "algorithmic": "4*D*sum_selected(n_q*n_k) = %.4g FLOP per launch" % flops_layer,
+                "mma_issued_flop_per_launch": issued,
+                "padding_waste": 1.0 - flops_layer / issued if issued else None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, fl = dynrad_oracle_sample(wl, 1, mode)
+        cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"1 of {wl.heads} heads of the {wl.name} layer, DynamicRad {mode} mask + attention, "
+                         f"{secs:.1f} s"}
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict({kk: vv for kk, vv in workload_config(wl, world, BH).items()
+                            if kk not in ("kmeans_iters", "top_p", "cq", "ck")},
+                           mask=f"DynamicRad {mode}", frames=frames, blocks=Cb, **DYNRAD),
+            "attn_ms": attn_ms, "attn_eff_tflops": flops_layer / (attn_ms * 1e-3) / 1e12,
+            "density": pairs / (BH * N * N),
+            "stages": {"mask": {"ms": mask_ms}, "attn": {"ms": attn_ms}},
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(3 * hq.numel() * 2),
+                    "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": (4 if mode == "dynamic" else 3) * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def load_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu capture, if it matches the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -523,6 +698,8 @@ def main(argv=None):
     ap.add_argument("--top-p", type=float, default=None, help="override the workload's (first) top-p")
     ap.add_argument("--kv-gather", type=int, default=0, choices=[0, 1],
                     help="1: no permuted K/V copies; the attention kernel gathers K/V rows through the K permutation")
+    ap.add_argument("--mask", default="svg2", choices=["svg2", "dynrad-static", "dynrad-dynamic"],
+                    help="block masks: SVG2 (k-means + top-p, the headline) or DynamicRad's two modes")
     ap.add_argument("--heads", type=int, default=None,
                     help="first H heads of the workload only (smaller case for profiler captures)")
     args = ap.parse_args(argv)
@@ -531,6 +708,8 @@ def main(argv=None):
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.mask != "svg2":
+        return run_dynrad(args, wl)
     return run_svg(args, wl)
 
 

@@ -209,6 +209,47 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
                                   void *o, float *lse, void *ws, size_t ws_bytes,
                                   svg_stream_t stream);
 
+/* ------------------------------------------------------------------------ DynamicRad block masks
+ * Block masks of the page "DynamicRad: Content-Adaptive Sparse Attention for
+ * Long Video Diffusion", section 2(a) (radial candidate set; static-ratio and
+ * dynamic-threshold modes), written in the block-list format of
+ * svg_select_topp so svg_sparse_attn runs them on Q, K and V in token order
+ * (q_off = k_off = offsets; no permutation).
+ *
+ * Tokens are frame-major: token n = t*S + s with S = N / frames.  A block is
+ * `block` consecutive tokens of one frame: a frame has nb = ceil(S / block)
+ * blocks (the last one ragged), block id c = t*nb + b.  Key block (t2, b2) is
+ * a candidate of query block (t1, b1) iff |b1 - b2| <= w(|t1 - t2|),
+ * w(d) = floor(w0 * gamma^d) (gamma^d formed by d successive float64
+ * multiplications).  Modes:
+ *   SVG_DYNRAD_CANDIDATES  every candidate;
+ *   SVG_DYNRAD_STATIC      per key frame the max(1, ceil(rho(d) * m)) candidates
+ *                          nearest to b1 (ties to the lower b2), m = candidates
+ *                          in that frame, rho(d) = min(1, rho0 * gamma^d);
+ *   SVG_DYNRAD_DYNAMIC     candidates whose proxy scale * mean(q rows of the
+ *                          query block) . mean(k rows of the key block)
+ *                          (float64) is >= theta; a query block keeping none
+ *                          keeps its highest-proxy candidate (ties: lower id).
+ *
+ *   q, k       [BH, N, D] bf16 (read in dynamic mode only; may be NULL otherwise)
+ *   offsets    [BH, Cb+1] int32  out: first token of every block, then N
+ *   sel_count  [BH, Cb]   int32  out: kept key blocks per query block (>= 1)
+ *   sel_cols   [BH, Cb, Cb] int32 out: kept key block ids, ascending
+ *   ws         dynamic mode: svg_dynrad_workspace_size bytes (the float64
+ *              block means); unused otherwise
+ * Cb = svg_dynrad_num_blocks(N, frames, block) (0 when frames does not divide
+ * N or an argument is not positive).  Requires Cb <= 1024
+ * (SVG_ERR_UNSUPPORTED), w0 >= 0, gamma >= 0, rho0 > 0 in static mode, and
+ * D = 64 or 128 in dynamic mode.  scale <= 0 selects 1/sqrt(D).
+ */
+enum { SVG_DYNRAD_CANDIDATES = 0, SVG_DYNRAD_STATIC = 1, SVG_DYNRAD_DYNAMIC = 2 };
+int svg_dynrad_num_blocks(int N, int frames, int block);
+size_t svg_dynrad_workspace_size(int BH, int N, int D, int frames, int block);
+svg_status svg_dynrad_select(const void *q, const void *k, int BH, int N, int D, int frames, int block, int mode,
+                             float w0, float gamma, float rho0, float theta, float scale, int32_t *offsets,
+                             int32_t *sel_count, int32_t *sel_cols, void *ws, size_t ws_bytes,
+                             svg_stream_t stream);
+
 /* ------------------------------------------------------------------------ sparse attention, no allocation
  * No counterpart on the pages: this is a service for callers that cannot hand
  * the library a scratch buffer.  Some callers have no way to obtain device

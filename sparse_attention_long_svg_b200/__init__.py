@@ -51,6 +51,9 @@ SIGNATURES = {
     "svg_sparse_attn_gather": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
                                     _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "svg_dynrad_num_blocks": (_I, [_I, _I, _I]),
+    "svg_dynrad_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "svg_dynrad_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _F, _F, _F, _P, _P, _P, _P, _SZ, _P]),
     "svg_sparse_attn_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P]),
     "svg_profile_enable": (_I, [_I]),
     "svg_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
@@ -303,6 +306,52 @@ def sparse_attn_gather(qp, k, v, perm_k, q_off, k_off, sel_count, sel_cols, scal
         _ptr(sel_cols), float(scale), _ptr(perm_q), _ptr(op), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return op, lse
+
+
+DYNRAD_MODES = {"candidates": 0, "static": 1, "dynamic": 2}
+
+
+def dynrad_select(q, k, frames: int, block: int, mode: str, w0: float, gamma: float, rho0: float = 1.0,
+                  theta: float = 0.0, scale: float = 0.0, offsets=None, sel_count=None, sel_cols=None,
+                  workspace=None, stream=None):
+    """DynamicRad block masks (svg_dynrad_select) for q, k [BH, N, D] bf16 in token order.
+
+    Returns (offsets [BH, Cb+1], sel_count [BH, Cb], sel_cols [BH, Cb, Cb]): the
+    block list svg_sparse_attn consumes with q_off = k_off = offsets.
+    """
+    lib = load_library()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k, "k", torch.bfloat16, 3)
+    BH, N, D = q.shape
+    Cb = lib.svg_dynrad_num_blocks(N, frames, block)
+    if Cb <= 0:
+        raise ValueError(f"frames {frames} must divide N {N} and block must be positive")
+    i32 = dict(dtype=torch.int32, device=q.device)
+    if offsets is None:
+        offsets = torch.empty((BH, Cb + 1), **i32)
+    if sel_count is None:
+        sel_count = torch.empty((BH, Cb), **i32)
+    if sel_cols is None:
+        sel_cols = torch.empty((BH, Cb, Cb), **i32)
+    if workspace is None:
+        workspace = _ws(lib.svg_dynrad_workspace_size(BH, N, D, frames, block), q.device)
+    _check("svg_dynrad_select", lib.svg_dynrad_select(
+        _ptr(q), _ptr(k), BH, N, D, int(frames), int(block), DYNRAD_MODES[mode], float(w0), float(gamma),
+        float(rho0), float(theta), float(scale), _ptr(offsets), _ptr(sel_count), _ptr(sel_cols), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return offsets, sel_count, sel_cols
+
+
+def dynrad_attention(q, k, v, frames: int, block: int, mode: str, w0: float, gamma: float, rho0: float = 1.0,
+                     theta: float = 0.0, scale: float = 0.0, out=None, want_lse: bool = False, stream=None):
+    """One attention layer with DynamicRad block masks (token order in and out, no permutation).
+
+    Returns (out, lse or None, (offsets, sel_count, sel_cols))."""
+    blocks = dynrad_select(q, k, frames, block, mode, w0, gamma, rho0, theta, scale, stream=stream)
+    offsets, sel_count, sel_cols = blocks
+    out, lse = sparse_attn(q, k, v, offsets, offsets, sel_count, sel_cols, scale, out, want_lse=want_lse,
+                           stream=stream)
+    return out, lse, blocks
 
 
 def sparse_attn_noalloc(qp, kp, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,

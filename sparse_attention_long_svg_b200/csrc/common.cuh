@@ -159,6 +159,13 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// Minimum of three floats in one instruction.
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int32_t x,
                                             int32_t y, uint64_t *bar) {

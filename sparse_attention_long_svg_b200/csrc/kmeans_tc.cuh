@@ -291,14 +291,17 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
     // Group g owns tile g of every pair; thread `row` = token n0 + row = TMEM
     // lane row.  Accumulators 2g and 2g + 1 alternate.
     //
-    // Best two centroids per row with three min/max operations per score.
+    // Best two centroids per row with five min/max operations per two scores.
     // Every score s becomes a key: s with its low byte replaced by the
     // column's position in its 64-column half-chunk (a change of at most
     // 2^-15 |s|), so the keys of one half-chunk are distinct and each names
-    // its column.  The half-chunk's two smallest keys follow
-    //   m2 = min(m2, max(m1, k)),  m1 = min(m1, k)
-    // in two interleaved chains, and are then merged into the running best
-    // and runner-up with the half-chunk's first column (an equal key keeps the
+    // its column.  The half-chunk's two smallest keys are kept in four
+    // independent chains (the chains are latency-bound, so more of them keep
+    // the ALU busy); a chain takes its keys two at a time:
+    //   lo = min(a, b), hi = max(a, b),
+    //   m2 = min(m2, hi, max(m1, lo)),  m1 = min(m1, lo).
+    // The chains are then merged pairwise and into the running best and
+    // runner-up with the half-chunk's first column (an equal key keeps the
     // earlier column, chunks are taken in ascending order).
     // Near-tie rule: a key is within 2^-15 |s| of its score, and the
     // tensor-core score is within about 2^-16 (||x||^2 + ||mu||^2) of the
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
         uint32_t buf[2][32];
         tmem_ld32_start(acc_addr, buf[0]);
         tmem_wait32(buf[0]);
-        float p1 = kBig, p2 = kBig, q1 = kBig, q2 = kBig;
+        float a1[4] = {kBig, kBig, kBig, kBig}, a2[4] = {kBig, kBig, kBig, kBig};   // four chains
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc) {
           if (pc < 3) {
@@ -361,21 +364,23 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 nv = __ldg(nv4 + pc * 8 + c4);
             const float nn[4] = {nv.x, nv.y, nv.z, nv.w};
+            float kk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float sc = fmaf(-2.f, __uint_as_float(acc[4 * c4 + e]), nn[e]);
-              const float kk = __int_as_float(
-                  __byte_perm(__float_as_int(sc), colb[(pc & 1) * 8 + c4], 0x3214 + e));
-              if (e & 1) {
-                q2 = fminf(q2, fmaxf(q1, kk));
-                q1 = fminf(q1, kk);
-              } else {
-                p2 = fminf(p2, fmaxf(p1, kk));
-                p1 = fminf(p1, kk);
-              }
+              kk[e] = __int_as_float(__byte_perm(__float_as_int(sc), colb[(pc & 1) * 8 + c4], 0x3214 + e));
+            }
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {   // chain (c4 & 1) * 2 + pr takes keys 2 pr, 2 pr + 1
+              const int ch = (c4 & 1) * 2 + pr;
+              const float lo = fminf(kk[2 * pr], kk[2 * pr + 1]), hi = fmaxf(kk[2 * pr], kk[2 * pr + 1]);
+              a2[ch] = min3f(a2[ch], hi, fmaxf(a1[ch], lo));
+              a1[ch] = fminf(a1[ch], lo);
             }
           }
-          if (pc & 1) {          // end of a 64-column half: merge its pair
+          if (pc & 1) {          // end of a 64-column half: merge the chains' pairs
+            const float p1 = fminf(a1[0], a1[1]), p2 = fminf(fmaxf(a1[0], a1[1]), fminf(a2[0], a2[1]));
+            const float q1 = fminf(a1[2], a1[3]), q2 = fminf(fmaxf(a1[2], a1[3]), fminf(a2[2], a2[3]));
             const float m1 = fminf(p1, q1);
             const float m2 = fminf(fmaxf(p1, q1), fminf(p2, q2));
             const int cbase = j * Cfg::NC + (pc >> 1) * 64;
@@ -388,7 +393,8 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
             arg = n1 ? mc1 : arg;
             second = ns;
             arg2 = nsa;
-            p1 = p2 = q1 = q2 = kBig;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) a1[ch] = a2[ch] = kBig;
           }
           if (pc < 3) tmem_wait32(buf[(pc + 1) & 1]);
         }

@@ -9,6 +9,7 @@
 
 #include "attn.cuh"
 #include "common.cuh"
+#include "dynrad.cuh"
 #include "kmeans.cuh"
 #include "kmeans_tc.cuh"
 #include "select.cuh"
@@ -619,6 +620,64 @@ svg_status svg_sparse_attn_unpermuted(const void *qp, const void *kp, const void
   if (!perm_q) return SVG_ERR_INVALID_ARG;
   return sparse_attn_impl(qp, kp, vp, nullptr, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols,
                           scale, perm_q, o, lse, ws, ws_bytes, stream);
+}
+
+int svg_dynrad_num_blocks(int N, int frames, int block) {
+  if (N <= 0 || frames <= 0 || block <= 0 || N % frames != 0) return 0;
+  const long long cb = static_cast<long long>(frames) * dynrad_blocks_per_frame(N, frames, block);
+  return cb > (1ll << 30) ? 0 : static_cast<int>(cb);
+}
+
+size_t svg_dynrad_workspace_size(int BH, int N, int D, int frames, int block) {
+  const int Cb = svg_dynrad_num_blocks(N, frames, block);
+  if (Cb == 0 || BH <= 0 || D <= 0 || !sizes_ok(BH, N)) return 0;
+  return align256(2ull * static_cast<size_t>(BH) * Cb * D * sizeof(double));
+}
+
+svg_status svg_dynrad_select(const void *q, const void *k, int BH, int N, int D, int frames, int block, int mode,
+                             float w0, float gamma, float rho0, float theta, float scale, int32_t *offsets,
+                             int32_t *sel_count, int32_t *sel_cols, void *ws, size_t ws_bytes,
+                             svg_stream_t stream) {
+  if (!offsets || !sel_count || !sel_cols || !sizes_ok(BH, N)) return SVG_ERR_INVALID_ARG;
+  const int Cb = svg_dynrad_num_blocks(N, frames, block);
+  if (Cb == 0) return SVG_ERR_INVALID_ARG;
+  if (Cb > kDynradMaxBlocks) return SVG_ERR_UNSUPPORTED;
+  if (mode < SVG_DYNRAD_CANDIDATES || mode > SVG_DYNRAD_DYNAMIC) return SVG_ERR_INVALID_ARG;
+  if (!(w0 >= 0.f) || !(gamma >= 0.f) || !(w0 < 1e30f) || !(gamma < 1e30f)) return SVG_ERR_INVALID_ARG;
+  if (mode == SVG_DYNRAD_STATIC && !(rho0 > 0.f && rho0 < 1e30f)) return SVG_ERR_INVALID_ARG;
+  const bool dynamic = mode == SVG_DYNRAD_DYNAMIC;
+  if (dynamic) {
+    if (!q || !k || !ws || std::isnan(theta)) return SVG_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(ws, 256)) return SVG_ERR_INVALID_ARG;
+    if (ws_bytes < svg_dynrad_workspace_size(BH, N, D, frames, block)) return SVG_ERR_WORKSPACE;
+  }
+  const int nb = dynrad_blocks_per_frame(N, frames, block);
+  const double scale_d = scale > 0.f ? static_cast<double>(scale) : 1.0 / std::sqrt(static_cast<double>(D));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n_off = BH * (Cb + 1);
+  dynrad_offsets_kernel<<<(n_off + 255) / 256, 256, 0, s>>>(BH, N, frames, nb, block, offsets);
+  if (launch_status("dynrad_offsets_kernel") != SVG_OK) return SVG_ERR_CUDA;
+  double *means = static_cast<double *>(ws);
+  const dim3 g(Cb, BH);
+  if (dynamic) {
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k);
+    if (D == 128)
+      dynrad_means_kernel<128><<<dim3(Cb, BH, 2), 128, 0, s>>>(qb, kb, BH, N, frames, nb, block, means);
+    else
+      dynrad_means_kernel<64><<<dim3(Cb, BH, 2), 64, 0, s>>>(qb, kb, BH, N, frames, nb, block, means);
+    if (launch_status("dynrad_means_kernel") != SVG_OK) return SVG_ERR_CUDA;
+  }
+  const int Dk = dynamic ? D : 64;   // the query-mean buffer is only read in dynamic mode
+  const size_t smem = dynrad_select_smem(frames, Dk);
+  const double w0d = w0, gd = gamma, rd = rho0, td = theta;
+  if (Dk == 128)
+    dynrad_select_kernel<128><<<g, 32, smem, s>>>(BH, frames, nb, mode, w0d, gd, rd, td, scale_d, means,
+                                                  sel_count, sel_cols);
+  else
+    dynrad_select_kernel<64><<<g, 32, smem, s>>>(BH, frames, nb, mode, w0d, gd, rd, td, scale_d,
+                                                 dynamic ? means : nullptr, sel_count, sel_cols);
+  return launch_status("dynrad_select_kernel");
 }
 
 svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, const int32_t *perm_k,

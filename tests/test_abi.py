@@ -62,6 +62,14 @@ def _p(v):
 FAKE = 0x10000  # 256-byte aligned, never dereferenced: every call below fails its host checks
 
 
+def test_dynrad_block_counts(lib):
+    assert lib.svg_dynrad_num_blocks(30, 3, 4) == 9          # frames of 10 tokens: blocks of 4, 4, 2
+    assert lib.svg_dynrad_num_blocks(32760, 21, 256) == 147  # 480p: 1,560 tokens per frame, 7 blocks
+    assert lib.svg_dynrad_num_blocks(31, 3, 4) == 0
+    assert lib.svg_dynrad_num_blocks(30, 3, 0) == 0
+    assert lib.svg_dynrad_workspace_size(40, 32760, 128, 21, 256) == 2 * 40 * 147 * 128 * 8
+
+
 def test_invalid_arguments_are_rejected_before_launch(lib):
     nul = _p(0)
     f = _p(FAKE)
@@ -97,5 +105,22 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
                                           8, nul) == 3
     # unpermute: aliasing
     assert lib.svg_unpermute(f, f, 1, 16, 64, f, nul) == 1
+    # gathered-K/V attention: missing perm_k, output aliasing K
+    assert lib.svg_sparse_attn_gather(f, f, f, nul, 1, 16, 64, f, 2, f, 2, f, f, 0.0, nul, g, nul, f,
+                                      1 << 20, nul) == 1
+    assert lib.svg_sparse_attn_gather(f, g, f, f, 1, 16, 64, f, 2, f, 2, f, f, 0.0, nul, g, nul, f,
+                                      1 << 20, nul) == 1
+    # DynamicRad masks: frames not dividing N, more than 1024 blocks, bad mode, negative window,
+    # static ratio <= 0, dynamic mode without q/k, unsupported D, small workspace
+    dyn = lambda q, N, D, fr, blk, mode, w0=2.0, gamma=0.5, rho0=0.5, ws=1 << 20: lib.svg_dynrad_select(
+        q, q, 1, N, D, fr, blk, mode, w0, gamma, rho0, 0.0, 0.0, f, f, f, f, ws, nul)
+    assert dyn(f, 30, 64, 4, 4, 1) == 1
+    assert dyn(f, 2048, 64, 1, 1, 1) == 2
+    assert dyn(f, 30, 64, 3, 4, 3) == 1
+    assert dyn(f, 30, 64, 3, 4, 1, w0=-1.0) == 1
+    assert dyn(f, 30, 64, 3, 4, 1, rho0=0.0) == 1
+    assert dyn(nul, 30, 64, 3, 4, 2) == 1
+    assert dyn(f, 30, 96, 3, 4, 2) == 2
+    assert dyn(f, 30, 64, 3, 4, 2, ws=8) == 3
     # nothing above reached CUDA
     assert lib.svg_last_cuda_error().decode() == ""
