@@ -20,13 +20,19 @@
 //     the CTA's units belong to the same head; only x streams (4-deep ring);
 //   * C > 128: consecutive tiles of one head are taken in pairs, and every
 //     chunk (hi and lo parts through a 4-deep ring) feeds both tiles' MMA
-//     chains before it is released, halving the centroid traffic per tile.
+//     chains before it is released, halving the centroid traffic per tile;
+//     a third x slot lets the next pair's first tile load while the current
+//     pair's last chunk is multiplied.
 // Warps 0-7: epilogue in two groups of four; group g owns tile g of every
 // pair (thread t of a group = token t of the tile = TMEM lane t) and keeps
 // the running best pair over all chunks of its tile, so the groups never
-// merge.  Warp 8: TMA producer.  Warp 9: MMA issuer and TMEM owner; each
-// (tile, chunk) is one chain of 2 x D/16 MMAs (hi then lo) into one of the
-// group's two TMEM accumulators.
+// merge.  Warp 8: TMA producer.  Warps 9 and 10: one MMA issuer per tile of
+// a pair (warp 9 owns TMEM); each (tile, chunk) is one chain of 2 x D/16 MMAs
+// (hi then lo) into one of the group's two TMEM accumulators.  The issuing
+// thread runs in step with the tensor pipe (a chain of 16 MMAs takes about as
+// long to issue as to execute), so with one issuer every barrier wait
+// between chains left the pipe idle; with two, one tile's chain executes
+// while the other issuer waits.
 #pragma once
 #include "common.cuh"
 
@@ -37,7 +43,7 @@ constexpr int kKmChunk = 128;   // centroids per chunk (MMA N)
 template <int D, bool SINGLE>
 struct KmCfg {
   static constexpr int BM = 128, NC = kKmChunk, DH = D / 64;
-  static constexpr int XST = SINGLE ? 4 : 2;   // x tile ring
+  static constexpr int XST = SINGLE ? 5 : 3;   // x tile ring (pairs: the next pair's first tile loads early)
   static constexpr int CST = SINGLE ? 2 : 4;   // centroid part ring (a part = hi or lo of a chunk)
   static constexpr int X_BYTES = BM * D * 2, C_BYTES = NC * D * 2;
   static constexpr int HALF = 128 * 128;       // one 64-channel half of a 128-row tile
@@ -49,12 +55,14 @@ struct KmCfg {
   static constexpr uint32_t TM_COLS = AST * NC;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, NC, false, false);
   static constexpr int EPI_WARPS = 8;          // two groups of four
-  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
-  static constexpr int PRODUCER_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
+  static constexpr int THREADS = (EPI_WARPS + 3) * 32;
+  static constexpr int PRODUCER_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1, MMA_B_WARP = EPI_WARPS + 2;
+  static_assert(XST <= 6 && CST <= 4, "barrier arrays");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
-struct KmBarriers {
-  uint64_t x_full[4], x_empty[4], c_full[4], c_empty[4], acc_full[4], acc_empty[4], drain;
+struct KmBarriers {   // x rings have at most 6 slots
+  uint64_t x_full[6], x_empty[6], c_full[4], c_empty[4], acc_full[4], acc_empty[4], drain[2];
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -136,15 +144,18 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
   const int u_end = static_cast<int>(units * (blockIdx.x + 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < Cfg::XST; ++s) {
       mbar_init(&B->x_full[s], 1);
-      mbar_init(&B->x_empty[s], 1);          // released by an MMA commit
+      mbar_init(&B->x_empty[s], 1);          // released by the epilogue (see there)
+    }
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&B->c_full[s], 1);
-      mbar_init(&B->c_empty[s], 1);
+      mbar_init(&B->c_empty[s], 2);          // both tiles' readers (see the MMA issuers)
       mbar_init(&B->acc_full[s], 1);
       mbar_init(&B->acc_empty[s], 4);        // the four warps of the group that read it
     }
-    mbar_init(&B->drain, 1);
+    mbar_init(&B->drain[0], 1);
+    mbar_init(&B->drain[1], 1);
     B->abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,10 +229,16 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
           mbar_wait(&B->c_full[k % Cfg::CST], (k / Cfg::CST) & 1, 1000000000ull);
       }
     }
-  } else if (warp == Cfg::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == Cfg::MMA_WARP || warp == Cfg::MMA_B_WARP) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer x takes tile x of every pair.  A commit covers only its own
+    // thread's MMAs, so the centroid parts of a chunk are released by both
+    // tiles' epilogue groups (c_empty counts two arrivals), and in the
+    // one-chunk case both issuers commit the resident chunk's release when
+    // the head changes.
+    const int x = warp == Cfg::MMA_WARP ? 0 : 1;
     if (lane == 0) {
-      uint32_t nx = 0, nc = 0, kacc[2] = {0, 0};
+      uint32_t nx = 0, nc = 0, kacc = 0;
       bool ok = true;
       int cur_h = -1;
       // descriptors of x slot 0 and centroid slot 0, built once; a slot adds its offset
@@ -243,24 +260,23 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
           nc += 2;
           cur_h = h;
         }
-        for (int j = 0; j < nchunks && ok; ++j) {
-          uint32_t c_hi = nc - 2, c_lo = nc - 1;   // SINGLE: the resident parts
-          if (!SINGLE) {
-            c_hi = nc;
-            c_lo = nc + 1;
-            if (!km_wait(B, &B->c_full[c_hi % Cfg::CST], (c_hi / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA) ||
-                !km_wait(B, &B->c_full[c_lo % Cfg::CST], (c_lo / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA)) {
-              ok = false;
-              break;
+        if (x < nt) {
+          const uint32_t xn = nx + x;
+          for (int j = 0; j < nchunks && ok; ++j) {
+            uint32_t c_hi = nc - 2, c_lo = nc - 1;   // SINGLE: the resident parts
+            if (!SINGLE) {
+              c_hi = nc + 2 * j;
+              c_lo = c_hi + 1;
+              if (!km_wait(B, &B->c_full[c_hi % Cfg::CST], (c_hi / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA) ||
+                  !km_wait(B, &B->c_full[c_lo % Cfg::CST], (c_lo / Cfg::CST) & 1, wait_ns, SITE_KMEANS_MMA)) {
+                ok = false;
+                break;
+              }
             }
-          }
-          for (int t = 0; t < nt; ++t) {
-            const uint32_t xn = nx + t;
-            const int ab = 2 * t + static_cast<int>(kacc[t] & 1);
+            const int ab = 2 * x + static_cast<int>(kacc & 1);
             if ((j == 0 && !km_wait(B, &B->x_full[xn % Cfg::XST], (xn / Cfg::XST) & 1, wait_ns,
                                     SITE_KMEANS_MMA)) ||
-                (kacc[t] >= 2 && !km_wait(B, &B->acc_empty[ab], ((kacc[t] >> 1) - 1) & 1, wait_ns,
-                                          SITE_KMEANS_MMA))) {
+                (kacc >= 2 && !km_wait(B, &B->acc_empty[ab], ((kacc >> 1) - 1) & 1, wait_ns, SITE_KMEANS_MMA))) {
               ok = false;
               break;
             }
@@ -270,21 +286,16 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
             const SmemDesc ld{cd0.lo + (((c_lo % Cfg::CST) * Cfg::C_BYTES) >> 4), cd0.hi};
             mma_chain<D / 16, Cfg::HALF, 32, Cfg::HALF, 32>(tmem + ab * Cfg::NC, xd, hd, Cfg::IDESC, 0u);
             mma_chain<D / 16, Cfg::HALF, 32, Cfg::HALF, 32>(tmem + ab * Cfg::NC, xd, ld, Cfg::IDESC, 1u);
-            mma_commit(&B->acc_full[ab]);
-            ++kacc[t];
-            if (j == nchunks - 1) mma_commit(&B->x_empty[xn % Cfg::XST]);   // last reader of this x tile
-          }
-          if (!SINGLE && ok) {
-            mma_commit(&B->c_empty[c_hi % Cfg::CST]);
-            mma_commit(&B->c_empty[c_lo % Cfg::CST]);
-            nc += 2;
+            mma_commit(&B->acc_full[ab]);   // the only commit of a chain (slots are released by the epilogue)
+            ++kacc;
           }
         }
+        if (!SINGLE) nc += 2 * nchunks;
         nx += nt;
         u += nt;
       }
-      mma_commit(&B->drain);
-      mbar_wait(&B->drain, 0, 1000000000ull);
+      mma_commit(&B->drain[x]);
+      mbar_wait(&B->drain[x], 0, 1000000000ull);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -320,11 +331,21 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
     for (int r = 0; r < 16; ++r)
       asm volatile("mov.b32 %0, %1;" : "=r"(colb[r]) : "r"(0x03020100u + 0x04040404u * r));
     uint32_t k = 0;   // accumulators this group has read
+    // Slot releases: an accumulator's commit tracks every earlier MMA of its
+    // issuer (one issuer per tile), so once a group sees the accumulator of
+    // its tile's last chunk, that tile's x slot is no longer read, and once
+    // it sees chunk j, its tile no longer reads chunk j's parts (c_empty
+    // counts both tiles).  The epilogue arrives on those barriers itself,
+    // which leaves one commit per MMA chain.
+    uint32_t nx_ep = 0, nc_ep = 0;   // x tiles and centroid parts of earlier pairs (the MMA issuer's counts)
     bool ok = true;
     for (int u0 = u_begin; u0 < u_end && ok; ) {
       const int nt = km_pair_tiles(u0, u_end, tiles);
       const int u = u0 + grp;
       u0 += nt;
+      const uint32_t xn_tile = nx_ep + grp, nc_pair = nc_ep;
+      nx_ep += nt;
+      if (!SINGLE) nc_ep += 2 * nchunks;
       if (grp >= nt) continue;
       const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
       const bool valid = n0 + row < N;
@@ -342,6 +363,15 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
           break;
         }
         tc_fence_after();
+        if (threadIdx.x == static_cast<unsigned>(grp * 128)) {   // one thread of the group
+          if (j == nchunks - 1) mbar_arrive(&B->x_empty[xn_tile % Cfg::XST]);
+          if (!SINGLE) {   // this tile no longer reads chunk j (the lone tile of a pair counts twice)
+            for (int r = 0; r < (nt == 1 ? 2 : 1); ++r) {
+              mbar_arrive(&B->c_empty[(nc_pair + 2 * j) % Cfg::CST]);
+              mbar_arrive(&B->c_empty[(nc_pair + 2 * j + 1) % Cfg::CST]);
+            }
+          }
+        }
         const float4 *nv4 = reinterpret_cast<const float4 *>(nh + j * Cfg::NC);
         const uint32_t acc_addr = tmem + lane_off + ab * Cfg::NC;
         // 32-column pieces: the next piece's TMEM load is in flight while the
