@@ -235,7 +235,7 @@ def workload_config(wl, n_gpus, heads=None, iters=None, top_p=None):
 
 def kernel_launches_per_step(iters: int) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
-    per_kmeans = 2 + 4 * iters               # split, |x|^2 + T x (assign, refine, bucket, accumulate)
+    per_kmeans = 1 + 4 * iters               # split + T x (assign, refine, bucket, accumulate); ||x||^2 in the first assign
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
     return 2 * per_kmeans + 2 * per_permute + 1 + 3       # select; plan x2 + attention (un-permute fused)
 

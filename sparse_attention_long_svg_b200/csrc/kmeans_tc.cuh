@@ -127,9 +127,9 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
                             const __grid_constant__ CUtensorMap map_hi,
                             const __grid_constant__ CUtensorMap map_lo, int BH, int N, int C,
                             int Cpad, const float *__restrict__ norms,
-                            const float *__restrict__ xnorm, int32_t *__restrict__ assign,
+                            float *__restrict__ xnorm, int32_t *__restrict__ assign,
                             int32_t *__restrict__ counts, KmTie *__restrict__ ties,
-                            int32_t *__restrict__ num_ties, uint64_t wait_ns) {
+                            int32_t *__restrict__ num_ties, int make_xnorm, uint64_t wait_ns) {
   using Cfg = KmCfg<D, SINGLE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::XST; ++s) {
       mbar_init(&B->x_full[s], 1);
-      mbar_init(&B->x_empty[s], 1);          // released by the epilogue (see there)
+      mbar_init(&B->x_empty[s], 4);          // released by the four epilogue warps of the tile's group
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(&B->c_full[s], 1);
@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
       const float *nh = norms + static_cast<size_t>(h) * Cpad;
       float best = kBig, second = kBig;
       int arg = 0x7fffffff, arg2 = -1;
+      float xx = 0.f;   // ||x||^2 of this row (first round: from the x tile in shared memory)
       for (int j = 0; j < nchunks; ++j, ++k) {
         const int ab = 2 * grp + static_cast<int>(k & 1);
         if (!__all_sync(0xffffffffu, mbar_wait(&B->acc_full[ab], (k >> 1) & 1, wait_ns))) {
@@ -364,13 +365,46 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
         }
         tc_fence_after();
         if (threadIdx.x == static_cast<unsigned>(grp * 128)) {   // one thread of the group
-          if (j == nchunks - 1) mbar_arrive(&B->x_empty[xn_tile % Cfg::XST]);
           if (!SINGLE) {   // this tile no longer reads chunk j (the lone tile of a pair counts twice)
             for (int r = 0; r < (nt == 1 ? 2 : 1); ++r) {
               mbar_arrive(&B->c_empty[(nc_pair + 2 * j) % Cfg::CST]);
               mbar_arrive(&B->c_empty[(nc_pair + 2 * j + 1) % Cfg::CST]);
             }
           }
+        }
+        if (make_xnorm && j == 0) {
+          // The x tile stays in its slot until this group releases it after
+          // the tile's last chunk; its own barrier (no later phase can have
+          // started) orders the copy before these reads.
+          if (!__all_sync(0xffffffffu, mbar_wait(&B->x_full[xn_tile % Cfg::XST], (xn_tile / Cfg::XST) & 1,
+                                                 wait_ns))) {
+            if (lane == 0) {
+              record_error(SVG_ERR_TIMEOUT, SITE_KMEANS_EPI);
+              atomicExch(&B->abort_flag, 1);
+            }
+            ok = false;
+            break;
+          }
+          const uint8_t *xr = smem + Cfg::OFF_X + (xn_tile % Cfg::XST) * Cfg::X_BYTES + row * 128;
+#pragma unroll
+          for (int dh = 0; dh < Cfg::DH; ++dh) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row sits at chunk c ^ (row % 8)
+              const uint4 v = *reinterpret_cast<const uint4 *>(xr + dh * Cfg::HALF + ((c ^ (row & 7)) << 4));
+              const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(b2[e]);
+                xx = fmaf(f.x, f.x, xx);
+                xx = fmaf(f.y, f.y, xx);
+              }
+            }
+          }
+          if (valid) xnorm[static_cast<size_t>(h) * N + n0 + row] = xx;
+        }
+        if (j == nchunks - 1) {   // every warp of the group is done with the x tile (x_empty counts four)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B->x_empty[xn_tile % Cfg::XST]);
         }
         const float4 *nv4 = reinterpret_cast<const float4 *>(nh + j * Cfg::NC);
         const uint32_t acc_addr = tmem + lane_off + ab * Cfg::NC;
@@ -434,7 +468,7 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
       if (valid && !live) record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);
       bool tie = false;
       if (live && arg2 >= 0 && arg2 < C) {
-        const float xx = __ldg(xnorm + static_cast<size_t>(h) * N + n0 + row);
+        if (!make_xnorm) xx = xnorm[static_cast<size_t>(h) * N + n0 + row];
         const float mm = fmaxf(__ldg(nh + arg), __ldg(nh + arg2));
         tie = second - best <= 0x1p-14f * (fabsf(best) + fabsf(second) + xx + mm);
       }
@@ -463,30 +497,6 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::TM_COLS);
   }
-}
-
-// ||x_n||^2 in fp32 for every token (x does not change across rounds); each
-// thread squares one 16-byte vector, the D/8 threads of a row add theirs.
-template <int D>
-__global__ void __launch_bounds__(256) kmeans_xnorm_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                           size_t tokens, float *__restrict__ xnorm) {
-  constexpr int VPR = D / 8;
-  const size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const size_t t = v / VPR;
-  float s = 0.f;
-  if (t < tokens) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x) + v);
-    const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(b2[e]);
-      s = fmaf(f.x, f.x, s);
-      s = fmaf(f.y, f.y, s);
-    }
-  }
-#pragma unroll
-  for (int o = VPR / 2; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (t < tokens && (threadIdx.x % VPR) == 0) xnorm[t] = s;
 }
 
 // Decides every listed near tie with the exact float32 distances

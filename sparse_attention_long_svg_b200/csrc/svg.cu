@@ -366,13 +366,8 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   kmeans_split_kernel<<<dim3((Cpad + 7) / 8, BH), 256, 0, s>>>(centroids, C, Cpad, D, w.hi, w.lo,
                                                               w.norms, w.num_ties, w.counters);
   if (launch_status("kmeans_split_kernel") != SVG_OK) return SVG_ERR_CUDA;
-  const size_t tokens = static_cast<size_t>(BH) * N;
-  const unsigned xnb = static_cast<unsigned>((tokens * (D / 8) + 255) / 256);
-  if (D == 128)
-    kmeans_xnorm_kernel<128><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
-  else
-    kmeans_xnorm_kernel<64><<<xnb, 256, 0, s>>>(xb, tokens, w.xnorm);
-  if (launch_status("kmeans_xnorm_kernel") != SVG_OK) return SVG_ERR_CUDA;
+  // ||x||^2 per token (for the near-tie margin) is formed by the first
+  // round's assign from the x tiles it loads anyway, and read by later rounds
   const int units = BH * ((N + 127) / 128);
   const int ga = units < num_sms() ? units : num_sms();
   const dim3 gb((N + 1024 * kBucketTokens - 1) / (1024 * kBucketTokens), BH);
@@ -381,10 +376,11 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   // one centroid chunk (C <= 128): the chunk stays resident per head; more:
   // tiles in pairs sharing every chunk
   const bool single = Cpad == kKmChunk;
+  int make_xnorm = 1;
   auto assign_kernel = [&](auto kernel, size_t smem_bytes, int threads) {
     if (!set_smem(kernel, smem_bytes)) return SVG_ERR_CUDA;
     kernel<<<ga, threads, smem_bytes, s>>>(mx, mhi, mlo, BH, N, C, Cpad, w.norms, w.xnorm, assign,
-                                          sizes, w.ties, w.num_ties, g_wait_ns);
+                                          sizes, w.ties, w.num_ties, make_xnorm, g_wait_ns);
     return launch_status("kmeans_assign_tc_kernel");
   };
   for (int it = 0; it < iters; ++it) {
@@ -402,6 +398,7 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
                   : assign_kernel(kmeans_assign_tc_kernel<64, false>, KmCfg<64, false>::SMEM_BYTES,
                                   KmCfg<64, false>::THREADS);
     if (st != SVG_OK) return st;
+    make_xnorm = 0;
     if (pe) cudaEventRecord(pe[1], s);
     if (D == 128)
       kmeans_refine_kernel<128><<<num_sms() * 4, 256, 0, s>>>(xb, N, C, centroids, w.ties,
