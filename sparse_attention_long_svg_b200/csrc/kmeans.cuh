@@ -187,12 +187,16 @@ __device__ __forceinline__ void kmeans_finalize_cluster(const double (&sum)[8], 
   }
 }
 
-// grid (ceil(max_accum_chunks(N, C) / 8), BH), 256 threads: warp w of block b
-// sums chunk j = 8 b + w.  A row is D/8 lanes x 16 bytes; a warp load covers
+// grid (ceil(max_accum_chunks(N, C) / kAccumWarps), BH), 32 kAccumWarps
+// threads: warp w of block b sums chunk j = kAccumWarps b + w.  One-warp blocks:
+// chunk lengths vary and a block holds its SM slot until its longest warp
+// ends.  A row is D/8 lanes x 16 bytes; a warp load covers
 // 32 / (D/8) rows, UNROLL loads are in flight.  Lane l keeps channels
 // 8 (l % (D/8)) .. +7 in fp64.
+constexpr int kAccumWarps = 1;
+
 template <int D>
-__global__ void __launch_bounds__(256) kmeans_accum_kernel(
+__global__ void __launch_bounds__(32 * kAccumWarps) kmeans_accum_kernel(
     const __nv_bfloat16 *__restrict__ x, int N, int C, int Cpad, const int32_t *__restrict__ bucket,
     const int32_t *__restrict__ offsets, const KmChunk *__restrict__ chunks,
     const int32_t *__restrict__ num_chunks, double *__restrict__ partial,
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(256) kmeans_accum_kernel(
   constexpr int STEP = RPL * UNROLL;   // rows per iteration
   const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + warp;
+  const int j = blockIdx.x * kAccumWarps + warp;
   if (j == 0 && h == 0 && lane == 0) *num_ties = 0;   // the refine step of this round is done
   if (j >= num_chunks[h]) return;
   const int maxch = max_accum_chunks(N, C);

@@ -371,7 +371,7 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   const int units = BH * ((N + 127) / 128);
   const int ga = units < num_sms() ? units : num_sms();
   const dim3 gb((N + 1024 * kBucketTokens - 1) / (1024 * kBucketTokens), BH);
-  const dim3 gacc((max_accum_chunks(N, C) + 7) / 8, BH);
+  const dim3 gacc((max_accum_chunks(N, C) + kAccumWarps - 1) / kAccumWarps, BH);
   int32_t *sizes = w.sizes(BH, C), *cursor = w.cursor(BH, C), *arrive = w.arrive(BH, C);
   // one centroid chunk (C <= 128): the chunk stays resident per head; more:
   // tiles in pairs sharing every chunk
@@ -411,11 +411,11 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
                                              counts, w.chunks, w.num_chunks);
     if (launch_status("kmeans_bucket_kernel") != SVG_OK) return SVG_ERR_CUDA;
     if (D == 128)
-      kmeans_accum_kernel<128><<<gacc, 256, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
+      kmeans_accum_kernel<128><<<gacc, 32 * kAccumWarps, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
                                                     w.num_chunks, w.partial, arrive, sizes, cursor,
                                                     centroids, w.hi, w.lo, w.norms, w.num_ties);
     else
-      kmeans_accum_kernel<64><<<gacc, 256, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
+      kmeans_accum_kernel<64><<<gacc, 32 * kAccumWarps, 0, s>>>(xb, N, C, Cpad, w.bucket, w.offsets, w.chunks,
                                                    w.num_chunks, w.partial, arrive, sizes, cursor,
                                                    centroids, w.hi, w.lo, w.norms, w.num_ties);
     if (launch_status("kmeans_accum_kernel") != SVG_OK) return SVG_ERR_CUDA;
