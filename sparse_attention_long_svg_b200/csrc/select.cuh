@@ -40,7 +40,7 @@ __device__ __forceinline__ uint64_t select_key(double w, int j) {
 
 // CPL = k-clusters per lane (ceil(Ck / 32) rounded up to 4, 8, 16 or 32).
 template <int D, int CPL>
-__global__ void __launch_bounds__(kSelRows * 32) select_topp_kernel(
+__global__ void __launch_bounds__(kSelRows * 32, CPL <= 16 ? 3 : 2) select_topp_kernel(
     const float *__restrict__ mu_q, const int32_t *__restrict__ n_q, const float *__restrict__ mu_k,
     const int32_t *__restrict__ n_k, int Cq, int Ck, float p, double scale,
     int32_t *__restrict__ sel_count, int32_t *__restrict__ sel_cols) {
