@@ -237,7 +237,7 @@ def kernel_launches_per_step(iters: int) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
     per_kmeans = 1 + 4 * iters               # split + T x (assign, refine, bucket, accumulate); ||x||^2 in the first assign
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
-    return 2 * per_kmeans + 2 * per_permute + 1 + 3       # select; plan x2 + attention (un-permute fused)
+    return 2 * per_kmeans + 2 * per_permute + 1 + 4       # select; plan x3 + attention (un-permute fused)
 
 
 def attention_pairs(layer, wl):
@@ -662,7 +662,7 @@ def run_dynrad(args, wl):
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(3 * hq.numel() * 2),
                     "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms / e2e_steps},
-            "gpu_launches": (4 if mode == "dynamic" else 3) * args.steps,
+            "gpu_launches": (6 if mode == "dynamic" else 5) * args.steps,   # mask (offsets, [means,] select) + plan x3 + attention
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -262,9 +262,9 @@ svg_status svg_dynrad_select(const void *q, const void *k, int BH, int N, int D,
  * every GPU which loads the library holds until the process exits.
  *
  *  - Limit: svg_sparse_attn_workspace_size(BH, N, Cq), about
- *    16*BH*(ceil(N/256) + Cq) + 8*BH*Cq bytes plus 2.5 MiB of per-CTA key
+ *    16*BH*(ceil(N/256) + Cq) + 16*BH*Cq bytes plus 2.5 MiB of per-CTA key
  *    ranges, must not exceed SVG_NOALLOC_SCRATCH_BYTES (e.g. 80 heads x 75,600
- *    tokens x 200 q-clusters needs 3.4 MB); larger sizes return
+ *    tokens x 200 q-clusters needs 3.5 MB); larger sizes return
  *    SVG_ERR_WORKSPACE before anything is launched.
  *  - It allocates and frees nothing (no cudaMalloc, no cudaFree, no
  *    allocating library routine).

@@ -54,7 +54,9 @@ constexpr int kItemRows = 256;     // query rows per work item (two 128-row tile
 constexpr int kSlotsPerTile = 16;  // 8-row slots per 128-key tile
 constexpr int kMetaRing = 8;       // key-validity masks in flight
 
-struct AttnItem {  // up to 256 query rows of one q-cluster; h < 0 ends the list
+struct AttnItem {  // up to 256 consecutive query rows; h < 0 ends the list
+  // i = the q-cluster whose block list the rows use (the rows may span a group
+  // of consecutive q-clusters with identical block lists)
   int32_t h, i, q0, packed;  // packed = rows (<= 256) | key_tiles << 9
 };
 
@@ -991,18 +993,55 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 }
 
 // ------------------------------------------------------------------ planning
+// Per (head, q-cluster): whether its block list equals the previous
+// q-cluster's (same non-empty count, same ids).  Such neighbours attend to the
+// same keys, so their consecutive permuted rows are planned as one row range:
+// the query tiles then pack rows of several clusters instead of padding each
+// cluster's tail.
+__global__ void attn_plan_merge_kernel(const int32_t *__restrict__ q_off, const int32_t *__restrict__ sel_count,
+                                       const int32_t *__restrict__ sel_cols, int BH, int Cq, int Ck, int max_sel,
+                                       int32_t *__restrict__ same_prev) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= BH * Cq) return;
+  const int h = idx / Cq, i = idx % Cq;
+  int same = 0;
+  if (i > 0) {
+    const int32_t *qo = q_off + h * (Cq + 1);
+    const int c0 = sel_count[idx - 1], c1 = sel_count[idx];
+    if (c0 == c1 && c1 > 0 && c1 <= max_sel && qo[i] > qo[i - 1] && qo[i + 1] > qo[i]) {
+      const int32_t *a = sel_cols + static_cast<size_t>(idx - 1) * Ck, *b = sel_cols + static_cast<size_t>(idx) * Ck;
+      same = 1;
+      for (int c = 0; c < c1 && same; ++c) same = a[c] == b[c];
+    }
+  }
+  same_prev[idx] = same;
+}
+
 // Per (head, q-cluster): number of work items (256 query rows each) and of
-// 128-key tiles per item.
+// 128-key tiles per item.  A q-cluster whose block list equals its
+// predecessor's has no items of its own: the first cluster of such a group
+// plans the group's rows (q_end = the group's last row + 1).
 __global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
                                        const int32_t *__restrict__ k_off,
                                        const int32_t *__restrict__ sel_count,
                                        const int32_t *__restrict__ sel_cols, int BH, int Cq, int Ck,
-                                       int max_sel, int32_t *__restrict__ qtiles,
-                                       int32_t *__restrict__ ktiles) {
+                                       int max_sel, const int32_t *__restrict__ same_prev,
+                                       int32_t *__restrict__ qtiles, int32_t *__restrict__ ktiles,
+                                       int32_t *__restrict__ q_end) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= BH * Cq) return;
   const int h = idx / Cq, i = idx % Cq;
-  const int nq = q_off[h * (Cq + 1) + i + 1] - q_off[h * (Cq + 1) + i];
+  if (same_prev[idx]) {   // planned by the first cluster of its group
+    qtiles[idx] = 0;
+    ktiles[idx] = 0;
+    q_end[idx] = 0;
+    return;
+  }
+  int last = i;
+  while (last + 1 < Cq && same_prev[idx + (last + 1 - i)]) ++last;
+  const int row_end = q_off[h * (Cq + 1) + last + 1];
+  q_end[idx] = row_end;
+  const int nq = row_end - q_off[h * (Cq + 1) + i];
   const int cnt = attn_sel_count(sel_count, idx, max_sel);
   const int32_t *cols = sel_cols + static_cast<size_t>(idx) * Ck;
   const int32_t *ko = k_off + static_cast<size_t>(h) * (Ck + 1);
@@ -1061,7 +1100,8 @@ __device__ __forceinline__ int attn_item_bucket(int h, int heads_per_group, int 
 
 __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
     const int32_t *__restrict__ q_off, const int32_t *__restrict__ qtiles,
-    const int32_t *__restrict__ ktiles, int BH, int Cq, AttnItem *__restrict__ items,
+    const int32_t *__restrict__ ktiles, const int32_t *__restrict__ q_end, int BH, int Cq,
+    AttnItem *__restrict__ items,
     int32_t *__restrict__ num_items, int32_t *__restrict__ next_item) {
   __shared__ int hist[kAttnBuckets];
   __shared__ int warp_tot[32];
@@ -1076,7 +1116,7 @@ __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
     if (qt <= 0) continue;
     const int kt = ktiles[idx];
     const int h = idx / Cq, i = idx % Cq;
-    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_off[h * (Cq + 1) + i + 1];
+    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_end[idx];
     for (int t = 0; t < qt; ++t)
       atomicAdd(&hist[attn_item_bucket(h, hpg, kt, min(kItemRows, row1 - row0 - t * kItemRows))], 1);
   }
@@ -1112,7 +1152,7 @@ __global__ void __launch_bounds__(1024) attn_plan_emit_kernel(
     if (qt <= 0) continue;
     const int kt = ktiles[idx];
     const int h = idx / Cq, i = idx % Cq;
-    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_off[h * (Cq + 1) + i + 1];
+    const int row0 = q_off[h * (Cq + 1) + i], row1 = q_end[idx];
     for (int t = 0; t < qt; ++t) {
       const int q0 = row0 + t * kItemRows;
       const int rows = min(kItemRows, row1 - q0);

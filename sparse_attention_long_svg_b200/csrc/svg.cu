@@ -142,7 +142,7 @@ KmeansWs carve_kmeans(void *ws, int BH, int N, int D, int C, size_t *bytes) {
 constexpr int kAttnMaxCtas = 160;
 
 struct AttnWs {
-  int32_t *num_items, *next_item, *qtiles, *ktiles;
+  int32_t *num_items, *next_item, *qtiles, *ktiles, *same_prev, *q_end;
   AttnItem *items;
   int2 *ranges;
 };
@@ -153,6 +153,8 @@ AttnWs carve_attn(void *ws, int BH, int N, int Cq, size_t *bytes) {
   w.next_item = c.take<int32_t>(1);
   w.qtiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.ktiles = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
+  w.same_prev = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
+  w.q_end = c.take<int32_t>(static_cast<size_t>(BH) * Cq);
   w.items = c.take<AttnItem>(static_cast<size_t>(BH) * ((N + kItemRows - 1) / kItemRows + Cq));
   w.ranges = c.take<int2>(static_cast<size_t>(kAttnMaxCtas) * 2 * AttnCfg<128>::MAX_SEL);
   *bytes = c.used;
@@ -535,9 +537,12 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
 
   const int pairs = BH * Cq;
   const int max_sel = Ck < AttnCfg<128>::MAX_SEL ? Ck : AttnCfg<128>::MAX_SEL;
+  attn_plan_merge_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, sel_count, sel_cols, BH, Cq, Ck, max_sel,
+                                                            w.same_prev);
   attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
-                                                            Cq, Ck, max_sel, w.qtiles, w.ktiles);
-  attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, BH, Cq, w.items,
+                                                            Cq, Ck, max_sel, w.same_prev, w.qtiles, w.ktiles,
+                                                            w.q_end);
+  attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, w.q_end, BH, Cq, w.items,
                                                    w.num_items, w.next_item);
   svg_status st = launch_status();
   if (st != SVG_OK) return st;

@@ -21,8 +21,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_launch_count_per_step():
     # per k-means call: split + |x|^2 + 4 per round; per permute: hist, scan, scatter, gather;
     # select; two planning kernels + attention (un-permute fused)
-    assert bench.kernel_launches_per_step(5) == 2 * (2 + 4 * 5) + 2 * 4 + 1 + 3 == 56
-    assert bench.kernel_launches_per_step(2) == 2 * (2 + 4 * 2) + 12
+    assert bench.kernel_launches_per_step(5) == 2 * (1 + 4 * 5) + 2 * 4 + 1 + 4 == 55
+    assert bench.kernel_launches_per_step(2) == 2 * (1 + 4 * 2) + 13
 
 
 def test_workload_config_keys():
