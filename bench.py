@@ -357,7 +357,6 @@ def run_svg(args, wl):
             step(events[s])
         t_end.record()
         torch.cuda.synchronize()
-    clocks.__exit__(None, None, None)
     assign_ms, assign_n, _ = svg.profile_read("kmeans_assign")
     attn_k_ms, attn_n, _ = svg.profile_read("sparse_attn")
     issued_pairs = svg.profile_attn_pairs()   # (128-row query tile, 128-key tile) pairs of the timed launches
@@ -370,6 +369,30 @@ def run_svg(args, wl):
         raise RuntimeError("device error word set during the timed steps: status %d at %s, CTA %d" % err)
     stage_ms = {n: statistics.mean(events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps))
                 for i, n in enumerate(stage_names)}
+    eager_ms = local_ms
+    if args.graph:
+        # the same layer step recorded once as a CUDA graph (centroid reset included) and replayed:
+        # one host launch per step instead of ~55, so no launch gaps between the kernels
+        graph = svg.LayerGraph(layer, q, k, v, mu_q0, mu_k0, T, p, 0.0, kv_gather=bool(args.kv_gather))
+        for _ in range(args.warmup):
+            graph.replay()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        local_ms = g0.elapsed_time(g1)
+        err = svg.get_error_detail()
+        if err[0] != 0:
+            raise RuntimeError("device error word set during the graph replays: status %d at %s, CTA %d" % err)
+        del graph
+    clocks.__exit__(None, None, None)   # the clock samples cover the eager and the graph-timed steps
 
     pairs = attention_pairs(layer, wl)
     flops_layer = 4.0 * D * pairs
@@ -489,6 +512,9 @@ def run_svg(args, wl):
                     "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": kernel_launches_per_step(T) * args.steps,
             "clocks": clocks.summary(),
+            "timing": ("CUDA-graph replays of the whole step (stages and per-kernel rooflines from eager steps "
+                       "with events; eager %.3f ms per step)" % (eager_ms / args.steps)) if args.graph else
+                      "eager launches",
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -696,6 +722,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="svg", choices=["svg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--top-p", type=float, default=None, help="override the workload's (first) top-p")
+    ap.add_argument("--graph", type=int, default=1, choices=[0, 1],
+                    help="1: time CUDA-graph replays of the whole layer step (0: eager launches)")
     ap.add_argument("--kv-gather", type=int, default=0, choices=[0, 1],
                     help="1: no permuted K/V copies; the attention kernel gathers K/V rows through the K permutation")
     ap.add_argument("--mask", default="svg2", choices=["svg2", "dynrad-static", "dynrad-dynamic"],

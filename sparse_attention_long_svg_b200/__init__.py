@@ -481,6 +481,44 @@ class SvgLayer:
                                self.kp, self.vp, op)
 
 
+class LayerGraph:
+    """One SvgLayer call recorded as a CUDA graph: replay() re-runs the whole layer
+    (k-means from the given initial centroids, permute, select, attention) on the
+    same device buffers with one launch from the host.
+
+    The captured call reads q, k, v and the initial centroids mu_q0 / mu_k0 from
+    the tensors given at capture time (refill them in place between replays) and
+    writes ``out``; mu_q / mu_k receive the final centroids.  The layer's own
+    kernels do no allocation and no host synchronisation, which is what makes
+    the capture valid.
+    """
+
+    def __init__(self, layer: "SvgLayer", q, k, v, mu_q0, mu_k0, iters: int, p: float, scale: float = 0.0,
+                 kv_gather: bool = False):
+        self.mu_q = torch.empty_like(mu_q0)
+        self.mu_k = torch.empty_like(mu_k0)
+        self.out = torch.empty_like(q)
+        args = (layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):        # one eager call: warms every kernel before capture
+            self._call(*args)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._call(*args)
+
+    def _call(self, layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather):
+        self.mu_q.copy_(mu_q0)
+        self.mu_k.copy_(mu_k0)
+        layer(q, k, v, self.mu_q, self.mu_k, iters, p, scale, self.out, kv_gather=kv_gather)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
+
+
 def svg_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mu_q: torch.Tensor, mu_k: torch.Tensor,
                   iters: int, p: float, scale: float = 0.0):
     """One SVG2 attention layer: returns (out [BH, N, D] bf16, LayerState).

@@ -294,6 +294,25 @@ def test_layer_kv_gather_equals_permuted_layer(name, case_data):
     assert torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("name", ["tiny", "small-d128"])
+def test_layer_graph_replay_equals_eager(name, case_data):
+    """The layer recorded as a CUDA graph and replayed gives the eager layer's output, bit for bit."""
+    L, _ = case_data(name)
+    H, N, D = L.q.shape
+    wl = L.workload
+    q, k, v = dev_bf16(L.q), dev_bf16(L.k), dev_bf16(L.v)
+    mq0, mk0 = dev_f32(L.init_centroids("q")), dev_f32(L.init_centroids("k"))
+    layer = svg.SvgLayer(H, N, D, wl.cq, wl.ck)
+    want, _ = layer(q, k, v, mq0.clone(), mk0.clone(), wl.iters, top_p_of(wl))
+    want = want.clone()
+    graph = svg.LayerGraph(layer, q, k, v, mq0, mk0, wl.iters, top_p_of(wl))
+    for _ in range(2):                       # replays start from the same initial centroids
+        got = graph.replay()
+        torch.cuda.synchronize()
+        assert svg.get_error() == 0
+        assert torch.equal(got, want)
+
+
 def test_sparse_attention_all_blocks_equals_dense(case_data):
     L, ref = case_data("tiny")
     H, N, D = L.q.shape
