@@ -233,11 +233,12 @@ def workload_config(wl, n_gpus, heads=None, iters=None, top_p=None):
 
 # ----------------------------------------------------------------------------- GPU leg
 
-def kernel_launches_per_step(iters: int) -> int:
+def kernel_launches_per_step(iters: int, qk_fp8: bool = False) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
     per_kmeans = 1 + 4 * iters               # split + T x (assign, refine, bucket, accumulate); ||x||^2 in the first assign
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
-    return 2 * per_kmeans + 2 * per_permute + 1 + 4       # select; plan x3 + attention (un-permute fused)
+    quant = (1 + 3) if qk_fp8 else 0         # Q per row; K per head: amax, quantise, scale
+    return 2 * per_kmeans + 2 * per_permute + 1 + quant + 4   # select; [quantise]; plan x3 + attention
 
 
 def attention_pairs(layer, wl):
@@ -300,6 +301,13 @@ def run_svg(args, wl):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
     stage_names = ["kmeans_q", "kmeans_k", "permute", "select", "attn+unpermute"]
+    if args.qk_fp8:
+        if args.kv_gather:
+            raise SystemExit("--qk-fp8 and --kv-gather cannot be combined")
+        q8 = torch.empty((BH, N, D), dtype=torch.float8_e4m3fn, device=device)
+        k8 = torch.empty_like(q8)
+        sq = torch.empty((BH, N), dtype=torch.float32, device=device)
+        sk = torch.empty((BH,), dtype=torch.float32, device=device)
 
     def step(ev=None):   # the un-permutation is fused into the attention kernel's store
         mu_q.copy_(mu_q0)
@@ -326,6 +334,11 @@ def run_svg(args, wl):
         if args.kv_gather:
             svg.sparse_attn_gather(layer.qp, k, v, layer.perm_k, layer.q_off, layer.k_off, layer.sel_count,
                                    layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
+        elif args.qk_fp8:        # E4M3 Q (per row) and K (per head), then attention with 8-bit Q K^T
+            svg.quantize_e4m3(layer.qp, True, q8, sq)
+            svg.quantize_e4m3(layer.kp, False, k8, sk)
+            svg.sparse_attn_fp8(q8, sq, k8, sk, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
+                                layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
         else:
             svg.sparse_attn(layer.qp, layer.kp, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
                             layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
@@ -373,7 +386,8 @@ def run_svg(args, wl):
     if args.graph:
         # the same layer step recorded once as a CUDA graph (centroid reset included) and replayed:
         # one host launch per step instead of ~55, so no launch gaps between the kernels
-        graph = svg.LayerGraph(layer, q, k, v, mu_q0, mu_k0, T, p, 0.0, kv_gather=bool(args.kv_gather))
+        graph = svg.LayerGraph(layer, q, k, v, mu_q0, mu_k0, T, p, 0.0, kv_gather=bool(args.kv_gather),
+                               qk_fp8=bool(args.qk_fp8))
         for _ in range(args.warmup):
             graph.replay()
         if world > 1:
@@ -422,7 +436,8 @@ def run_svg(args, wl):
         dv.copy_(hv, non_blocking=True)
         mu_q.copy_(hmq, non_blocking=True)
         mu_k.copy_(hmk, non_blocking=True)
-        o, _ = layer(dq, dk, dv, mu_q, mu_k, T, p, 0.0, out, kv_gather=bool(args.kv_gather))
+        o, _ = layer(dq, dk, dv, mu_q, mu_k, T, p, 0.0, out, kv_gather=bool(args.kv_gather),
+                     qk_fp8=bool(args.qk_fp8))
         hout.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
@@ -444,10 +459,19 @@ def run_svg(args, wl):
     attn_kernel_ms = attn_k_ms / max(attn_n, 1)
     attn_kernel_tflops = flops_layer / (attn_kernel_ms * 1e-3) / 1e12
     issued = issued_flops / max(attn_n, 1)
-    roof_attn = {"kernel": f"sparse_attn_kernel<{D}>", "bound": "tensor", "achieved": attn_kernel_tflops,
-                 "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_kernel_tflops / tc_peak,
-                 "frac_of_sustained": attn_kernel_tflops / tc_sust,
-                 "traffic": load_traffic("sparse_attn_kernel", wl.name), "peak_kind": peak_note,
+    attn_peak, attn_sust, attn_note, attn_name = tc_peak, tc_sust, peak_note, f"sparse_attn_kernel<{D}>"
+    if args.qk_fp8:
+        # half the FLOPs (S = Q K^T) at the E4M3 rate, half (P V) at the bf16 rate: with E4M3 at 2x bf16
+        # (the nominal ratio, applied to the measured bf16 peak) the ideal time is 3/4 of all-bf16
+        attn_peak, attn_sust = tc_peak * 4.0 / 3.0, tc_sust * 4.0 / 3.0
+        attn_note = ("4/3 x the " + peak_note + " (Q K^T on E4M3 at 2x the bf16 rate, P V on bf16)")
+        attn_name = f"sparse_attn_kernel<{D}, fp8 QK^T>"
+    roof_attn = {"kernel": attn_name, "bound": "tensor", "achieved": attn_kernel_tflops,
+                 "peak": attn_peak, "unit": "TFLOP/s", "frac": attn_kernel_tflops / attn_peak,
+                 "frac_of_sustained": attn_kernel_tflops / attn_sust,
+                 "frac_of_bf16_peak": attn_kernel_tflops / tc_peak,
+                 "traffic": load_traffic("sparse_attn_kernel_fp8" if args.qk_fp8 else "sparse_attn_kernel", wl.name),
+                 "peak_kind": attn_note,
                  "launch_ms": attn_kernel_ms, "launches": attn_n, "total_ms": attn_k_ms,
                  "algorithmic": "4*D*sum_selected(n_q*n_k) = %.4g FLOP per launch" % flops_layer,
                  "mma_issued_flop_per_launch": issued,
@@ -501,16 +525,19 @@ def run_svg(args, wl):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 QK^T, bf16 PV" if args.qk_fp8 else "bf16",
+            "data": "synthetic",
             "config": dict(workload_config(wl, world, BH, T, p),
                            kv=("gathered by the attention kernel through the K permutation" if args.kv_gather
-                               else "permuted copies written by svg_permute")),
+                               else "permuted copies written by svg_permute"),
+                           **({"qk": "E4M3 Q (per-row scales) and K (per-head scales), quantised each step"}
+                              if args.qk_fp8 else {})),
             "attn_ms": stage_ms["attn+unpermute"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,
             "roofline": roofline, "roofline_other": roofline_other, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / e2e_steps},
-            "gpu_launches": kernel_launches_per_step(T) * args.steps,
+            "gpu_launches": kernel_launches_per_step(T, bool(args.qk_fp8)) * args.steps,
             "clocks": clocks.summary(),
             "timing": ("CUDA-graph replays of the whole step (stages and per-kernel rooflines from eager steps "
                        "with events; eager %.3f ms per step)" % (eager_ms / args.steps)) if args.graph else
@@ -726,6 +753,8 @@ def main(argv=None):
                     help="1: time CUDA-graph replays of the whole layer step (0: eager launches)")
     ap.add_argument("--kv-gather", type=int, default=0, choices=[0, 1],
                     help="1: no permuted K/V copies; the attention kernel gathers K/V rows through the K permutation")
+    ap.add_argument("--qk-fp8", type=int, default=0, choices=[0, 1],
+                    help="1: Q and K quantised to E4M3 after the permutation; S = Q K^T on 8-bit tensor cores")
     ap.add_argument("--mask", default="svg2", choices=["svg2", "dynrad-static", "dynrad-dynamic"],
                     help="block masks: SVG2 (k-means + top-p, the headline) or DynamicRad's two modes")
     ap.add_argument("--heads", type=int, default=None,

@@ -209,6 +209,38 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
                                   void *o, float *lse, void *ws, size_t ws_bytes,
                                   svg_stream_t stream);
 
+/* ------------------------------------------------------------------------ 8-bit Q K^T
+ * Low-bit attention in the spirit of the page "TurboDiffusion" (section
+ * "SageAttention: low-bit quantization": attention on quantised operands to
+ * cut memory traffic and compute).  The page fixes no format; here Q and K
+ * are FP8 E4M3 (bias 7, 3 mantissa bits, largest finite 448; round to
+ * nearest, ties to even, saturating at +-448), the logits are
+ * scale * (q8 . k8) * s_q[row] * s_k[head], and P and V stay bf16.
+ *
+ * svg_quantize_e4m3: x [BH, N, D] bf16 -> x8 [BH, N, D] E4M3 bytes and float32
+ * scales, x8 = E4M3(x / s) with the division in float32 and
+ * s = amax|x| / 448 (1 where amax is 0):
+ *   per_row = 1   one scale per row, scales [BH * N]   (for Q)
+ *   per_row = 0   one scale per head over all N*D values, scales [BH]  (for K)
+ * D = 64 or 128.  x and x8 16-byte aligned, not aliased.  The per-head form
+ * zeroes `scales` (stream-ordered) before reducing into it.
+ *
+ * svg_sparse_attn_fp8: svg_sparse_attn / svg_sparse_attn_unpermuted with
+ * q8 [BH, N, D] and k8 [BH, N, D] E4M3 (permuted, as svg_quantize_e4m3 makes
+ * them from qp and kp), q_scale [BH * N] and k_scale [BH] their scales, vp
+ * bf16.  perm_q optional: with it o (and lse) are in token order, else in
+ * the Q-permuted order.  D must be 128 (SVG_ERR_UNSUPPORTED otherwise).  The
+ * workspace is svg_sparse_attn_workspace_size(BH, N, Cq) bytes; other
+ * arguments and the error behaviour are those of svg_sparse_attn.
+ */
+svg_status svg_quantize_e4m3(const void *x, int BH, int N, int D, int per_row, void *x8, float *scales,
+                             svg_stream_t stream);
+svg_status svg_sparse_attn_fp8(const void *q8, const float *q_scale, const void *k8, const float *k_scale,
+                               const void *vp, int BH, int N, int D, const int32_t *q_off, int Cq,
+                               const int32_t *k_off, int Ck, const int32_t *sel_count, const int32_t *sel_cols,
+                               float scale, const int32_t *perm_q, void *o, float *lse, void *ws,
+                               size_t ws_bytes, svg_stream_t stream);
+
 /* ------------------------------------------------------------------------ DynamicRad block masks
  * Block masks of the page "DynamicRad: Content-Adaptive Sparse Attention for
  * Long Video Diffusion", section 2(a) (radial candidate set; static-ratio and

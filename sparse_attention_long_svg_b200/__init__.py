@@ -51,6 +51,9 @@ SIGNATURES = {
     "svg_sparse_attn_gather": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
                                     _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "svg_quantize_e4m3": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "svg_sparse_attn_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P, _SZ,
+                                 _P]),
     "svg_dynrad_num_blocks": (_I, [_I, _I, _I]),
     "svg_dynrad_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "svg_dynrad_select": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _F, _F, _F, _P, _P, _P, _P, _SZ, _P]),
@@ -308,6 +311,53 @@ def sparse_attn_gather(qp, k, v, perm_k, q_off, k_off, sel_count, sel_cols, scal
     return op, lse
 
 
+def quantize_e4m3(x, per_row: bool, x8=None, scales=None, stream=None):
+    """E4M3 copy of x [BH, N, D] bf16 and its float32 scales (svg_quantize_e4m3):
+    per_row -> scales [BH, N] (one per row, for Q), else [BH] (one per head, for K).
+    Returns (x8 as torch.float8_e4m3fn, scales)."""
+    lib = load_library()
+    _need(x, "x", torch.bfloat16, 3)
+    BH, N, D = x.shape
+    if x8 is None:
+        x8 = torch.empty((BH, N, D), dtype=torch.float8_e4m3fn, device=x.device)
+    if scales is None:
+        scales = torch.empty((BH, N) if per_row else (BH,), dtype=torch.float32, device=x.device)
+    _check("svg_quantize_e4m3", lib.svg_quantize_e4m3(_ptr(x), BH, N, D, 1 if per_row else 0, _ptr(x8),
+                                                      _ptr(scales), _stream(stream)))
+    return x8, scales
+
+
+def sparse_attn_fp8(q8, q_scale, k8, k_scale, vp, q_off, k_off, sel_count, sel_cols, scale: float = 0.0, op=None,
+                    want_lse: bool = False, lse=None, workspace=None, stream=None, perm_q=None):
+    """Attention over the selected blocks with E4M3 Q and K (quantize_e4m3 of the
+    permuted qp, per row, and kp, per head) and bf16 V.  With ``perm_q`` the output
+    (and lse) come back in token order.  Returns (op, lse or None)."""
+    lib = load_library()
+    _need(q8, "q8", torch.float8_e4m3fn, 3)
+    _need(k8, "k8", torch.float8_e4m3fn, 3)
+    _need(vp, "vp", torch.bfloat16, 3)
+    BH, N, D = q8.shape
+    if q_scale.dtype != torch.float32 or q_scale.numel() != BH * N or not q_scale.is_contiguous():
+        raise ValueError("q_scale must be a contiguous float32 tensor of BH * N values")
+    if k_scale.dtype != torch.float32 or k_scale.numel() != BH or not k_scale.is_contiguous():
+        raise ValueError("k_scale must be a contiguous float32 tensor of BH values")
+    Cq = q_off.shape[1] - 1
+    Ck = k_off.shape[1] - 1
+    if op is None:
+        op = torch.empty((BH, N, D), dtype=torch.bfloat16, device=q8.device)
+    if want_lse and lse is None:
+        lse = torch.empty((BH, N), dtype=torch.float32, device=q8.device)
+    if workspace is None:
+        workspace = _ws(lib.svg_sparse_attn_workspace_size(BH, N, Cq), q8.device)
+    if perm_q is not None:
+        _need(perm_q, "perm_q", torch.int32, 2)
+    _check("svg_sparse_attn_fp8", lib.svg_sparse_attn_fp8(
+        _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(vp), BH, N, D, _ptr(q_off), Cq, _ptr(k_off), Ck,
+        _ptr(sel_count), _ptr(sel_cols), float(scale), _ptr(perm_q), _ptr(op), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return op, lse
+
+
 DYNRAD_MODES = {"candidates": 0, "static": 1, "dynamic": 2}
 
 
@@ -438,13 +488,18 @@ class SvgLayer:
                  lib.svg_permute_workspace_size(BH, N, max(Cq, Ck)),
                  lib.svg_sparse_attn_workspace_size(BH, N, Cq))
         self.workspace = _ws(ws, device)
+        self.fp8 = None     # (q8, q_scale, k8, k_scale), made by the first call with qk_fp8
 
     def __call__(self, q, k, v, mu_q, mu_k, iters: int, p: float, scale: float = 0.0, out=None, stream=None,
-                 fused_unpermute: bool = True, kv_gather: bool = False):
+                 fused_unpermute: bool = True, kv_gather: bool = False, qk_fp8: bool = False):
         """One layer; with ``fused_unpermute`` the attention kernel stores rows in token order
         (no permuted output copy, ``LayerState.op`` is None), else attention + svg_unpermute.
         With ``kv_gather`` K and V are not permuted: the attention kernel fetches their rows
-        through the K permutation (``LayerState.kp``/``vp`` are None); requires fused_unpermute."""
+        through the K permutation (``LayerState.kp``/``vp`` are None); requires fused_unpermute.
+        With ``qk_fp8`` the permuted Q and K are quantised to E4M3 (per-row / per-head scales)
+        and S = Q K^T runs on 8-bit operands; D must be 128."""
+        if qk_fp8 and kv_gather:
+            raise ValueError("qk_fp8 and kv_gather cannot be combined")
         kmeans(q, mu_q, iters, self.assign_q, self.n_q, self.workspace, stream)
         kmeans(k, mu_k, iters, self.assign_k, self.n_k, self.workspace, stream)
         Cq, Ck = mu_q.shape[1], mu_k.shape[1]
@@ -465,7 +520,28 @@ class SvgLayer:
             return out, LayerState(mu_q, mu_k, self.assign_q, self.assign_k, self.n_q, self.n_k, self.perm_q,
                                    self.perm_k, self.q_off, self.k_off, self.sel_count, self.sel_cols, self.qp,
                                    None, None, None)
-        if fused_unpermute:
+        if qk_fp8:
+            if self.fp8 is None:
+                BH, N, D = self.qp.shape
+                f8 = dict(dtype=torch.float8_e4m3fn, device=self.qp.device)
+                f32 = dict(dtype=torch.float32, device=self.qp.device)
+                self.fp8 = (torch.empty((BH, N, D), **f8), torch.empty((BH, N), **f32),
+                            torch.empty((BH, N, D), **f8), torch.empty((BH,), **f32))
+            q8, sq, k8, sk = self.fp8
+            quantize_e4m3(self.qp, True, q8, sq, stream)
+            quantize_e4m3(self.kp, False, k8, sk, stream)
+            if fused_unpermute:
+                if out is None:
+                    out = torch.empty_like(q)
+                sparse_attn_fp8(q8, sq, k8, sk, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols,
+                                scale, out, workspace=self.workspace, stream=stream, perm_q=self.perm_q)
+                op = None
+            else:
+                sparse_attn_fp8(q8, sq, k8, sk, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols,
+                                scale, self.op, workspace=self.workspace, stream=stream)
+                out = unpermute(self.op, self.perm_q, out, stream)
+                op = self.op
+        elif fused_unpermute:
             if out is None:
                 out = torch.empty_like(q)
             sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,
@@ -494,11 +570,11 @@ class LayerGraph:
     """
 
     def __init__(self, layer: "SvgLayer", q, k, v, mu_q0, mu_k0, iters: int, p: float, scale: float = 0.0,
-                 kv_gather: bool = False):
+                 kv_gather: bool = False, qk_fp8: bool = False):
         self.mu_q = torch.empty_like(mu_q0)
         self.mu_k = torch.empty_like(mu_k0)
         self.out = torch.empty_like(q)
-        args = (layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather)
+        args = (layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather, qk_fp8)
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):        # one eager call: warms every kernel before capture
@@ -509,10 +585,10 @@ class LayerGraph:
         with torch.cuda.graph(self.graph):
             self._call(*args)
 
-    def _call(self, layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather):
+    def _call(self, layer, q, k, v, mu_q0, mu_k0, iters, p, scale, kv_gather, qk_fp8):
         self.mu_q.copy_(mu_q0)
         self.mu_k.copy_(mu_k0)
-        layer(q, k, v, self.mu_q, self.mu_k, iters, p, scale, self.out, kv_gather=kv_gather)
+        layer(q, k, v, self.mu_q, self.mu_k, iters, p, scale, self.out, kv_gather=kv_gather, qk_fp8=qk_fp8)
 
     def replay(self):
         self.graph.replay()

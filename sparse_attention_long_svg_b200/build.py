@@ -33,6 +33,7 @@ def sources():
 KERNEL_SOURCES = {
     "kmeans_assign_tc_kernel": ("common.cuh", "kmeans_tc.cuh"),
     "sparse_attn_kernel": ("common.cuh", "attn.cuh"),
+    "sparse_attn_kernel_fp8": ("common.cuh", "attn.cuh"),
 }
 
 

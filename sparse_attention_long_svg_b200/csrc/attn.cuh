@@ -39,7 +39,9 @@
 // so one tile's exponentials overlap the other tile's MMAs; the turns also
 // let both tiles share one P buffer in shared memory (bf16, 128-byte
 // swizzled, K-major): P_x(t) is written once the previous PV (the other
-// tile's) has read it.  O accumulates in TMEM across the item's key tiles;
+// tile's) has read it.  With 8-bit Q and K (E4M3 Q K^T, kind::f8f6f4) the
+// smaller Q/K tiles leave room for one P buffer per query tile, and P_x(t)
+// waits only for PV_x(t-1).  O accumulates in TMEM across the item's key tiles;
 // the softmax warps rescale it in place only when a row's running max grows
 // by more than 2^8 (exact: every probability is taken against the same
 // reference max that O and the row sum use).  The merged key ranges of the
@@ -64,29 +66,76 @@ struct AttnItem {  // up to 256 consecutive query rows; h < 0 ends the list
 // the producer, the two MMA issuers and the eight softmax warps.
 constexpr int kItemReaders = 11;
 
-template <int D>
+// Instruction descriptor for kind::f8f6f4 with E4M3 A/B (format code 0 in
+// both operand fields), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7) | (0u << 10)                    // A, B format: E4M3
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+// D[tmem] (+)= A * B^T with 8-bit operands (kind::f8f6f4): one MMA covers 32
+// elements (32 bytes) of K.  Descriptors as halves plus 16-byte offsets.
+__device__ __forceinline__ void mma_f8_ss_off(uint32_t d_tmem, SmemDesc a, uint32_t a_off, SmemDesc b,
+                                              uint32_t b_off, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+      "mov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a.lo + a_off), "r"(a.hi), "r"(b.lo + b_off), "r"(b.hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The 8-bit counterpart of mma_chain: STEPS MMAs of 32 bytes of K each, K-step
+// k at byte offset k * 32 of a 128-byte swizzle row (STEPS <= 4).
+template <int STEPS, uint32_t A_K, uint32_t B_K>
+__device__ __forceinline__ void mma_chain_f8(uint32_t d_tmem, SmemDesc a, SmemDesc b, uint32_t idesc,
+                                             uint32_t accumulate_first) {
+  static_assert(STEPS <= 4, "one 128-byte block of K");
+#pragma unroll
+  for (int k = 0; k < STEPS; ++k)
+    mma_f8_ss_off(d_tmem, a, (k * A_K) >> 4, b, (k * B_K) >> 4, idesc, k > 0 ? 1u : accumulate_first);
+}
+
+// FP8: Q and K are E4M3 (one byte per channel, a 128-channel row is one
+// 128-byte swizzle row) and S = Q K^T runs as kind::f8f6f4 MMAs; P and V stay
+// bf16.  Supported at D = 128.
+template <int D, bool FP8 = false>
 struct AttnCfg {
   static constexpr int BM = 128, BN = 128, SLOT = 8, NSLOT = BN / SLOT;
   static constexpr int HEAD_DIM = D;
-  static constexpr int DH = D / 64;                   // 64-channel (128-byte) halves
+  static constexpr int QE = FP8 ? 1 : 2;              // bytes per Q/K element
+  static constexpr int QK_BLOCK = 128 / QE;           // Q/K channels per 128-byte block
+  static constexpr int DHQ = D * QE / 128;            // 128-byte blocks of a Q/K row
+  static constexpr int DH = D / 64;                   // 128-byte (64-channel) blocks of a V row
   static constexpr int KST = D == 128 ? 2 : 4;        // K ring slots (same for V)
-  static constexpr int QT_BYTES = BM * D * 2;         // one Q tile
-  static constexpr int KV_BYTES = BN * D * 2;         // one K or V tile
-  static constexpr int HALF_Q = BM * 128;             // one 64-channel half of a Q tile
-  static constexpr int HALF_KV = BN * 128;            // same for a K/V tile
-  static constexpr int P_BYTES = BM * BN * 2;         // the shared P tile
+  static constexpr int QT_BYTES = BM * D * QE;        // one Q tile
+  static constexpr int K_BYTES = BN * D * QE;         // one K tile
+  static constexpr int V_BYTES = BN * D * 2;          // one V tile
+  static constexpr int HALF_Q = BM * 128;             // one 128-byte column block of a Q tile
+  static constexpr int HALF_K = BN * 128;             // same for a K tile
+  static constexpr int HALF_V = BN * 128;             // same for a V tile
+  static constexpr int P_BYTES = BM * BN * 2;         // one P tile
   static constexpr int HALF_P = BM * 128;             // one 64-key half of it
+  // P buffers: one shared by both query tiles, or (FP8, whose 8-bit Q and K
+  // tiles leave the room) one per query tile
+  static constexpr int NP = FP8 ? 2 : 1;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = OFF_Q + 2 * QT_BYTES;
-  static constexpr int OFF_K = OFF_P + P_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_K = OFF_P + NP * P_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * K_BYTES;
   static constexpr int MAX_SEL = 1024;                // selected k-clusters per q-cluster
-  static constexpr int OFF_BAR = OFF_V + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + KST * V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers/meta + alignment slack
   // TMEM: S of tile x at x*128 (128 columns); O of tile x at 256 + x*128
   static constexpr uint32_t TM_COLS = 512;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+  static constexpr uint32_t IDESC_S =
+      FP8 ? idesc_e4m3_f32(BM, BN, false, false) : idesc_bf16_f32(BM, BN, false, false);
+  static constexpr int S_STEPS = D * QE / 32;         // MMAs of one S chain (32 bytes of K each)
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+  static_assert(!FP8 || D == 128, "8-bit Q/K tiles need 128-byte rows");
   // warp 9 issues tile A's MMAs (and owns TMEM), warp 11 tile B's
   static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, LOADER_WARP = 10, MMA_B_WARP = 11;
   static constexpr int THREADS = 12 * 32;
@@ -134,6 +183,7 @@ struct AttnBarriers {
   int32_t ranges_cnt[2]; // merged runs of the item in header slot [b]
   uint32_t meta[kMetaRing][4];   // per key tile: 128-bit key validity mask
   uint32_t exp_steps[2]; // [tile]: 4 x the steps whose exponentials that tile has finished (one add per warp)
+  uint32_t v_seen;       // two P buffers: V tiles whose landing tile A's MMA issuer has seen (all tiles, in order)
   uint32_t tmem_base;
   int32_t abort_flag;
 };
@@ -148,6 +198,8 @@ struct AttnParams {
   const int32_t *perm;   // optional: write row r of a head to row perm[r] (un-permuted output)
   const int32_t *perm_k; // gather mode: permuted key row r of a head is row perm_k[r] of K and V
   const __nv_bfloat16 *kg, *vg;   // gather mode: K and V [BH, N, D] in token order
+  const float *q_scale;  // FP8: per permuted query row [BH, N]; the logits carry q_scale * k_scale
+  const float *k_scale;  // FP8: per head [BH]
   unsigned long long *issued;   // optional: += (query tile, key tile) pairs issued
   int2 *ranges;          // per CTA: 2 x MAX_SEL merged key runs (first row, rows), one slot per header slot
   int N, Cq, Ck, BH;
@@ -208,6 +260,24 @@ __device__ __forceinline__ bool attn_warp_wait_count(AttnBarriers *b, const uint
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// One thread waits until a shared-memory progress counter reaches `target`
+// (wrap-safe comparison), bounded like the barrier waits.
+__device__ __forceinline__ bool attn_wait_count(AttnBarriers *b, const uint32_t *ctr, uint32_t target, uint64_t ns,
+                                                uint32_t site) {
+  const volatile uint32_t *c = ctr;
+  if (static_cast<int32_t>(*c - target) >= 0) return true;
+  const long long t0 = clock64();
+  const long long limit = static_cast<long long>(ns) * 2;
+  while (static_cast<int32_t>(*c - target) < 0) {
+    if (clock64() - t0 > limit) {
+      record_error(SVG_ERR_TIMEOUT, site);
+      atomicExch(&b->abort_flag, 1);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Number of selected k-clusters of a block-list row, clamped to [0, limit];
 // a count outside that range is recorded as a device check failure.
 __device__ __forceinline__ int attn_sel_count(const int32_t *sel_count, size_t row, int limit) {
@@ -221,7 +291,7 @@ __device__ __forceinline__ int attn_sel_count(const int32_t *sel_count, size_t r
 
 // Gather mode: one 128-row key tile (K or V) into a ring slot, in the same
 // 128-byte-swizzled K-major layout the tensor-map loads produce (row r,
-// 16-byte chunk c of 64-channel half h at h * HALF_KV + 128 r + 16 (c ^ r % 8)).
+// 16-byte chunk c of 64-channel half h at h * HALF_V + 128 r + 16 (c ^ r % 8)).
 // Lane l holds the global rows of tile rows 4 l .. 4 l + 3 in `rows`; each
 // warp instruction copies D / 8 consecutive 16-byte chunks of 32 / (D / 8)
 // rows (coalesced), the rows taken from their owners by shuffles.
@@ -231,7 +301,7 @@ __device__ __forceinline__ void gather_rows(uint32_t slot_addr, const __nv_bfloa
   constexpr int LPR = Cfg::HEAD_DIM / 8;   // lanes (16-byte chunks) per row
   constexpr int RPI = 32 / LPR;        // rows per instruction
   const int sub = lane / LPR, c = lane % LPR;
-  const uint32_t half_off = static_cast<uint32_t>((c >> 3) * Cfg::HALF_KV);
+  const uint32_t half_off = static_cast<uint32_t>((c >> 3) * Cfg::HALF_V);
   const int cc = c & 7;
 #pragma unroll
   for (int i = 0; i < Cfg::BN / RPI; ++i) {
@@ -254,10 +324,11 @@ __device__ __forceinline__ void gather_rows(uint32_t slot_addr, const __nv_bfloa
   }
 }
 
-template <int D, bool GATHER>
-__global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
+template <int D, bool GATHER, bool FP8 = false>
+__global__ void __launch_bounds__(AttnCfg<D, FP8>::THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams P) {
-  using Cfg = AttnCfg<D>;
+  using Cfg = AttnCfg<D, FP8>;
+  static_assert(!(GATHER && FP8), "gather mode copies bf16 rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -286,6 +357,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       mbar_init(&B->p_full[x], 4);
       mbar_init(&B->q_full[x], 1);
       B->exp_steps[x] = 0;
+      B->v_seen = 0;
       mbar_init(&B->o_full[x], 1);
       mbar_init(&B->item_full[x], 1);
       mbar_init(&B->item_empty[x], kItemReaders);
@@ -341,8 +413,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         break;
       }
       const AttnItem it = P.items[w];
-      if (lane < 2 * Cfg::DH && (lane / Cfg::DH) * Cfg::BM < (it.packed & 0x1FF))   // query rows -> L2
-        tma_prefetch_l2_2d(&maps.q, (lane % Cfg::DH) * 64, it.h * P.N + it.q0 + (lane / Cfg::DH) * Cfg::BM);
+      if (lane < 2 * Cfg::DHQ && (lane / Cfg::DHQ) * Cfg::BM < (it.packed & 0x1FF))   // query rows -> L2
+        tma_prefetch_l2_2d(&maps.q, (lane % Cfg::DHQ) * Cfg::QK_BLOCK,
+                           it.h * P.N + it.q0 + (lane / Cfg::DHQ) * Cfg::BM);
       const size_t row = static_cast<size_t>(it.h) * P.Cq + it.i;
       const int cnt = attn_sel_count(P.sel_count, row, max_sel);
       const int32_t *cols = P.sel_cols + row * P.Ck;
@@ -469,8 +542,8 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                 if (x == 1 && !has_b) break;
                 mbar_arrive_expect_tx(&B->q_full[x], Cfg::QT_BYTES);
 #pragma unroll
-                for (int dh = 0; dh < Cfg::DH; ++dh)
-                  tma_load_2d(sQ + x * Cfg::QT_BYTES + dh * Cfg::HALF_Q, &maps.q, dh * 64,
+                for (int dh = 0; dh < Cfg::DHQ; ++dh)
+                  tma_load_2d(sQ + x * Cfg::QT_BYTES + dh * Cfg::HALF_Q, &maps.q, dh * Cfg::QK_BLOCK,
                               qrow + x * Cfg::BM, &B->q_full[x]);
               }
             }
@@ -557,7 +630,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                 for (int w = 0; w < 4; ++w) B->meta[mi][w] = pre_mask[w];
                 mbar_arrive(&B->meta_full[mi]);
               }
-              gather_rows<Cfg>(smem_u32(sK + slot * Cfg::KV_BYTES), P.kg, r4, lane);
+              gather_rows<Cfg>(smem_u32(sK + slot * Cfg::K_BYTES), P.kg, r4, lane);
               cp_async_arrive(&B->k_full[slot]);
             } else {
               // cut the tile into boxes of 1..16 slots (8..128 rows): the largest
@@ -608,15 +681,15 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
   #pragma unroll
                 for (int w = 0; w < 4; ++w) B->meta[mi][w] = mask[w];
                 mbar_arrive(&B->meta_full[mi]);
-                mbar_arrive_expect_tx(&B->k_full[slot], Cfg::KV_BYTES);
+                mbar_arrive_expect_tx(&B->k_full[slot], Cfg::K_BYTES);
               }
               __syncwarp();
               if (my_code >= 0) {
                 const int kind = my_code & 0xFF, at = my_code >> 8;
   #pragma unroll
-                for (int dh = 0; dh < Cfg::DH; ++dh)
-                  tma_load_2d(sK + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.k[kind], dh * 64,
-                              my_row, &B->k_full[slot]);
+                for (int dh = 0; dh < Cfg::DHQ; ++dh)
+                  tma_load_2d(sK + slot * Cfg::K_BYTES + dh * Cfg::HALF_K + at * 1024, &maps.k[kind],
+                              dh * Cfg::QK_BLOCK, my_row, &B->k_full[slot]);
               }
             }
             ++gk;
@@ -648,7 +721,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
 #pragma unroll
               for (int e = 1; e < kBoxRing; ++e)
                 if (e == rb) r4 = grow[e];
-              gather_rows<Cfg>(smem_u32(sV + slot * Cfg::KV_BYTES), P.vg, r4, lane);
+              gather_rows<Cfg>(smem_u32(sV + slot * Cfg::V_BYTES), P.vg, r4, lane);
               cp_async_arrive(&B->v_full[slot]);
             } else {
               int my_row = -1, my_code = -1;
@@ -659,13 +732,13 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
                   my_code = box_code[e];
                 }
               }
-              if (lane == 0) mbar_arrive_expect_tx(&B->v_full[slot], Cfg::KV_BYTES);
+              if (lane == 0) mbar_arrive_expect_tx(&B->v_full[slot], Cfg::V_BYTES);
               __syncwarp();
               if (my_code >= 0) {
                 const int kind = my_code & 0xFF, at = my_code >> 8;
   #pragma unroll
                 for (int dh = 0; dh < Cfg::DH; ++dh)
-                  tma_load_2d(sV + slot * Cfg::KV_BYTES + dh * Cfg::HALF_KV + at * 1024, &maps.v[kind], dh * 64,
+                  tma_load_2d(sV + slot * Cfg::V_BYTES + dh * Cfg::HALF_V + at * 1024, &maps.v[kind], dh * 64,
                               my_row, &B->v_full[slot]);
               }
             }
@@ -714,9 +787,9 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const int x = warp == Cfg::MMA_WARP ? 0 : 1;
     if (lane == 0) {
       const SmemDesc qd = make_desc_sw128(smem_u32(sQ) + x * Cfg::QT_BYTES, 16, 1024);
-      const SmemDesc pd = make_desc_sw128(smem_u32(sP), 16, 1024);
+      const SmemDesc pd = make_desc_sw128(smem_u32(sP) + (Cfg::NP == 2 ? x * Cfg::P_BYTES : 0), 16, 1024);
       const SmemDesc kd0 = make_desc_sw128(smem_u32(sK), 16, 1024);
-      const SmemDesc vd0 = make_desc_sw128(smem_u32(sV), Cfg::HALF_KV, 1024);
+      const SmemDesc vd0 = make_desc_sw128(smem_u32(sV), Cfg::HALF_V, 1024);
       uint32_t g0 = 0, n_s = 0, n_pv = 0, n_q = 0;   // key tiles of earlier items; S, PV chains issued; Q tiles used
       unsigned long long pairs = 0;
       for (uint32_t n = 0; !aborted(B); ++n) {
@@ -740,7 +813,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
           const uint32_t gt = g0 + t;
           const int slot = static_cast<int>(gt % Cfg::KST);
           const uint32_t ph = (gt / Cfg::KST) & 1;
-          const uint32_t slot_off = (slot * Cfg::KV_BYTES) >> 4;
+          const uint32_t k_off = (slot * Cfg::K_BYTES) >> 4, v_off = (slot * Cfg::V_BYTES) >> 4;
           if (is_s) {
             if (!attn_wait(B, &B->k_full[slot], ph, ns, SITE_ATTN_MMA) ||
                 (n_s > 0 && !attn_wait(B, &B->s_free[x], (n_s - 1) & 1, ns, SITE_ATTN_MMA))) {
@@ -749,24 +822,36 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
             }
             if constexpr (GATHER) fence_proxy_async_smem();   // cp.async writes -> tensor-core reads
             tc_fence_after();
-            mma_chain<D / 16, Cfg::HALF_Q, 32, Cfg::HALF_KV, 32>(
-                tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + slot_off, kd0.hi}, Cfg::IDESC_S, 0u);
+            if constexpr (FP8)
+              mma_chain_f8<Cfg::S_STEPS, 32, 32>(tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + k_off, kd0.hi},
+                                                 Cfg::IDESC_S, 0u);
+            else
+              mma_chain<Cfg::S_STEPS, Cfg::HALF_Q, 32, Cfg::HALF_K, 32>(
+                  tmem + Cfg::tm_s(x), qd, SmemDesc{kd0.lo + k_off, kd0.hi}, Cfg::IDESC_S, 0u);
             mma_commit(&B->s_full[x]);
             mma_commit(&B->k_empty[x][slot]);
             if (t == ntk - 1) mma_commit(&B->q_empty[x]);   // the item's last S: Q may be replaced
             ++n_s;
           } else {
+            // with two P buffers tile B's P write no longer waits for tile A's
+            // PV; its first V wait of an item then waits first for tile A to
+            // have seen every earlier V tile land, so the slot barrier is at
+            // most one phase behind the awaited one
             if (!attn_wait(B, &B->p_full[x], n_pv & 1, ns, SITE_ATTN_MMA) ||
+                (Cfg::NP == 2 && x == 1 && t == 0 && !attn_wait_count(B, &B->v_seen, g0, ns, SITE_ATTN_MMA)) ||
                 !attn_wait(B, &B->v_full[slot], ph, ns, SITE_ATTN_MMA)) {
               ok = false;
               break;
+            }
+            if constexpr (Cfg::NP == 2) {
+              if (x == 0) *reinterpret_cast<volatile uint32_t *>(&B->v_seen) = gt + 1;
             }
             if constexpr (GATHER) fence_proxy_async_smem();
             tc_fence_after();
             // A = P [128 q x 128 keys], K-major in two 64-key halves; B = V [128 keys x D],
             // MN-major, 16 keys = 2048 bytes per K-step
             mma_chain<Cfg::BN / 16, Cfg::HALF_P, 32, 4 * 2048, 2048>(
-                tmem + Cfg::tm_o(x), pd, SmemDesc{vd0.lo + slot_off, vd0.hi}, Cfg::IDESC_PV, t > 0 ? 1u : 0u);
+                tmem + Cfg::tm_o(x), pd, SmemDesc{vd0.lo + v_off, vd0.hi}, Cfg::IDESC_PV, t > 0 ? 1u : 0u);
             mma_commit(&B->p_free[x]);                     // the shared P buffer may be rewritten
             if (t == ntk - 1) mma_commit(&B->o_full[x]);   // the item's O of tile x is final
             mma_commit(&B->v_empty[x][slot]);
@@ -795,7 +880,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t o_addr = tmem + lane_off + Cfg::tm_o(x);
     const uint32_t s_addr = tmem + lane_off + Cfg::tm_s(x);
-    const float sl2 = P.scale_log2;
+    float sl2 = P.scale_log2;   // FP8: times this row's Q scale and the head's K scale (set per item)
     uint32_t g = 0, n_s = 0, n_o = 0;
     // Exponentials take turns between the two tiles (A(t), B(t), A(t+1), ...),
     // so one tile's exponentials overlap the other tile's MMAs instead of
@@ -827,6 +912,12 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
       const int rows_total = it.packed & 0x1FF;
       const int nrows = x == 0 ? min(rows_total, Cfg::BM) : rows_total - Cfg::BM;
       const bool pair = rows_total > Cfg::BM;   // both tiles present: take turns
+      if constexpr (FP8) {
+        if (nrows > 0) {
+          const size_t gq = static_cast<size_t>(it.h) * P.N + it.q0 + x * Cfg::BM + row;
+          sl2 = P.scale_log2 * (row < nrows ? __ldg(P.q_scale + gq) : 1.f) * __ldg(P.k_scale + it.h);
+        }
+      }
       if (nrows <= 0) {          // this item has no tile B
         g += ntk;
         other_before += ntk;     // tile A's steps of this item
@@ -895,12 +986,17 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) atomicAdd(&B->exp_steps[x], 1u);
-        // the shared P buffer is free once the PV of the previous write has
-        // completed; that PV was issued after PV_x(t - 1) completed, so O_x
-        // is stable too
+        // a P buffer is free once the PV of its previous write has completed
+        // (shared buffer: that PV was issued after PV_x(t - 1) completed, so
+        // O_x is stable too; a buffer per tile: it is PV_x(t - 1) itself)
         int py = -1;              // tile whose PV read P last, and that PV's index
         uint32_t pidx = 0;
-        if (x == 1) {
+        if constexpr (Cfg::NP == 2) {   // own buffer: free once this tile's previous PV has completed
+          if (pv_before[x] + t > 0) {
+            py = x;
+            pidx = pv_before[x] + t - 1;
+          }
+        } else if (x == 1) {
           py = 0;
           pidx = pv_before[0] + t;                          // A(t)
         } else if (t > 0) {
@@ -930,7 +1026,7 @@ __global__ void __launch_bounds__(AttnCfg<D>::THREADS, 1)
         // 16-byte chunks XOR row % 8)
 #pragma unroll
         for (int kh = 0; kh < 2; ++kh) {
-          uint8_t *prow = sP + kh * Cfg::HALF_P + row * 128;
+          uint8_t *prow = sP + (Cfg::NP == 2 ? x * Cfg::P_BYTES : 0) + kh * Cfg::HALF_P + row * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint32_t chunk = u ^ (row & 7);

@@ -1,0 +1,157 @@
+// E4M3 quantisation of Q and K for the 8-bit Q K^T path of the attention
+// kernel.  The page "TurboDiffusion" (section "SageAttention: low-bit
+// quantization") runs attention on low-bit quantised operands to cut memory
+// traffic and compute; it fixes no format or scale rule.  Here:
+//   * E4M3 values (4 exponent bits, bias 7, 3 mantissa bits, largest finite
+//     448), rounded to nearest with ties to even, saturating at +-448;
+//   * Q: one float32 scale per token row, s = amax|row| / 448 (1 for an
+//     all-zero row); K: one float32 scale per head over all its rows, so a key
+//     tile gathered from any rows of the head shares it;
+//   * the stored value is E4M3(x / s), the division in float32.
+// The logits become scale * (q8 . k8) * s_q * s_k; P and V stay bf16.
+#pragma once
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace svg {
+
+constexpr float kE4m3Max = 448.f;
+
+__device__ __forceinline__ float e4m3_scale(float amax) {
+  return amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.f;
+}
+
+__device__ __forceinline__ uint32_t e4m3_byte(float v, float s) {
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Per-row scales: each lane converts 8 consecutive channels (one 16-byte
+// load); the D / 8 lanes of a row reduce its amax with shuffles, so a warp
+// covers 256 / D rows per pass, and two passes are in flight per iteration.
+template <int D>
+__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const __nv_bfloat16 *__restrict__ x, size_t rows,
+                                                              uint8_t *__restrict__ x8, float *__restrict__ scales) {
+  constexpr int LPR = D / 8;           // lanes per row
+  constexpr int RPW = 32 / LPR;        // rows per warp pass
+  constexpr int U = 2;                 // passes per iteration
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, c = lane % LPR;
+  const size_t warp = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const size_t warps = static_cast<size_t>(gridDim.x) * (blockDim.x >> 5);
+  for (size_t r0 = warp * (RPW * U); r0 < rows; r0 += warps * (RPW * U)) {
+    uint4 u[U];
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const size_t r = r0 + i * RPW + sub;
+      u[i] = r < rows ? __ldcs(reinterpret_cast<const uint4 *>(x + r * D) + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < U; ++i) {
+      const size_t r = r0 + i * RPW + sub;
+      const uint32_t w[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[j]);
+        v[2 * j] = __low2float(b);
+        v[2 * j + 1] = __high2float(b);
+      }
+      float m = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float s = e4m3_scale(m);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        lo |= e4m3_byte(v[e], s) << (8 * e);
+        hi |= e4m3_byte(v[4 + e], s) << (8 * e);
+      }
+      if (r < rows) {
+        reinterpret_cast<uint2 *>(x8 + r * D)[c] = make_uint2(lo, hi);
+        if (c == 0) scales[r] = s;
+      }
+    }
+  }
+}
+
+// Per-head amax: blocks (chunk, head) reduce 8-channel groups of the head's
+// N * D values and fold their maximum into amax_bits[head] (float bits of a
+// non-negative value order like integers; amax_bits is zero on entry).
+__global__ void __launch_bounds__(256) head_amax_kernel(const __nv_bfloat16 *__restrict__ x, size_t per_head,
+                                                        int32_t *__restrict__ amax_bits) {
+  const int h = blockIdx.y;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(h) * per_head);
+  const size_t groups = per_head / 8;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  float m = 0.f;
+  for (size_t g0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g0 < groups; g0 += 4 * stride) {
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const size_t g = g0 + k * stride;
+      u[k] = g < groups ? __ldcs(src + g) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+        m = fmaxf(m, fmaxf(fabsf(__low2float(b)), fabsf(__high2float(b))));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) b = fmaxf(b, wmax[w]);
+    atomicMax(amax_bits + h, __float_as_int(b));
+  }
+}
+
+// Quantises each head with the scale of its amax (read from amax_bits).
+__global__ void __launch_bounds__(256) quant_heads_e4m3_kernel(const __nv_bfloat16 *__restrict__ x, size_t per_head,
+                                                               const int32_t *__restrict__ amax_bits,
+                                                               uint8_t *__restrict__ x8) {
+  const int h = blockIdx.y;
+  const float s = e4m3_scale(__int_as_float(amax_bits[h]));
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(h) * per_head);
+  uint2 *dst = reinterpret_cast<uint2 *>(x8 + static_cast<size_t>(h) * per_head);
+  const size_t groups = per_head / 8;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t g0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g0 < groups; g0 += 2 * stride) {
+    uint4 u[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const size_t g = g0 + k * stride;
+      u[k] = g < groups ? __ldcs(src + g) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      uint32_t out[2] = {0, 0};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+        out[i >> 1] |= (e4m3_byte(__low2float(b), s) | (e4m3_byte(__high2float(b), s) << 8)) << (16 * (i & 1));
+      }
+      const size_t g = g0 + k * stride;
+      if (g < groups) dst[g] = make_uint2(out[0], out[1]);
+    }
+  }
+}
+
+// amax_bits[h] (float bits) -> scale[h], in place.
+__global__ void head_scale_kernel(int32_t *amax_bits, int BH) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h < BH) reinterpret_cast<float *>(amax_bits)[h] = e4m3_scale(__int_as_float(amax_bits[h]));
+}
+
+}  // namespace svg

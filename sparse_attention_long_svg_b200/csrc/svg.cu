@@ -10,6 +10,7 @@
 #include "attn.cuh"
 #include "common.cuh"
 #include "dynrad.cuh"
+#include "fp8.cuh"
 #include "kmeans.cuh"
 #include "kmeans_tc.cuh"
 #include "select.cuh"
@@ -58,18 +59,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// 2-D view [rows, D] of a bf16 tensor; boxes of 64 channels x box_rows rows,
-// 128-byte swizzle (the tcgen05 K-major / MN-major canonical layout).
-bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, int D, int box_rows) {
+// 2-D view [rows, D] of a bf16 (or, with u8, a one-byte-per-channel)
+// tensor; boxes of 128 bytes of channels x box_rows rows, 128-byte swizzle
+// (the tcgen05 K-major / MN-major canonical layout).
+bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, int D, int box_rows, bool u8 = false) {
   auto enc = encoder();
   if (!enc) return false;
+  const int eb = u8 ? 1 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * eb};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -512,19 +516,24 @@ size_t svg_sparse_attn_workspace_size(int BH, int N, int Cq) {
 }  // extern "C"
 
 namespace {
-// Shared body of svg_sparse_attn (perm == nullptr: permuted output rows) and
-// svg_sparse_attn_unpermuted (row r of a head stored at row perm[r]).
+// Shared body of svg_sparse_attn (perm == nullptr: permuted output rows),
+// svg_sparse_attn_unpermuted (row r of a head stored at row perm[r]),
+// svg_sparse_attn_gather (perm_k set) and svg_sparse_attn_fp8 (q_scale and
+// k_scale set: qp and kp hold E4M3 bytes).
 svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, const int32_t *perm_k,
                             int BH, int N, int D, const int32_t *q_off, int Cq, const int32_t *k_off,
                             int Ck, const int32_t *sel_count, const int32_t *sel_cols, float scale,
                             const int32_t *perm, void *op, float *lse, void *ws, size_t ws_bytes,
-                            svg_stream_t stream) {
+                            svg_stream_t stream, const float *q_scale = nullptr, const float *k_scale = nullptr) {
   if (!qp || !kp || !vp || !q_off || !k_off || !sel_count || !sel_cols || !op || !ws)
     return SVG_ERR_INVALID_ARG;
   const bool gather = perm_k != nullptr;
+  const bool fp8 = q_scale != nullptr;
+  if (fp8 && (k_scale == nullptr || gather)) return SVG_ERR_INVALID_ARG;
   if (perm != nullptr && (op == qp || op == kp || op == vp)) return SVG_ERR_INVALID_ARG;
   if (!sizes_ok(BH, N) || Cq < 1 || Ck < 1) return SVG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (fp8 && D != 128) return SVG_ERR_UNSUPPORTED;
   if (Ck > AttnCfg<128>::MAX_SEL) return SVG_ERR_UNSUPPORTED;
   if (!aligned(qp, 16) || !aligned(kp, 16) || !aligned(vp, 16) || !aligned(op, 16) ||
       !aligned(ws, 256))
@@ -550,9 +559,9 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
   AttnMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const uint64_t rows = static_cast<uint64_t>(BH) * N;
-  if (!make_map_bf16(&maps.q, qp, rows, D, 128)) return SVG_ERR_CUDA;
+  if (!make_map_bf16(&maps.q, qp, rows, D, 128, fp8)) return SVG_ERR_CUDA;
   for (int b = 0; b < (gather ? 0 : kNumBoxSizes); ++b)   // gather mode copies rows without tensor maps
-    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b) || !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
+    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b, fp8) || !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
       return SVG_ERR_CUDA;
   AttnParams prm;
   prm.q_off = q_off;
@@ -568,6 +577,8 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
   prm.perm_k = perm_k;
   prm.kg = static_cast<const __nv_bfloat16 *>(kp);
   prm.vg = static_cast<const __nv_bfloat16 *>(vp);
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
   prm.ranges = w.ranges;
   prm.issued = nullptr;
   if (g_prof.on) {
@@ -590,7 +601,9 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
     return true;
   };
   bool ok;
-  if (D == 128)
+  if (fp8)
+    ok = launch(sparse_attn_kernel<128, false, true>, AttnCfg<128, true>::THREADS, AttnCfg<128, true>::SMEM_BYTES);
+  else if (D == 128)
     ok = gather ? launch(sparse_attn_kernel<128, true>, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES)
                 : launch(sparse_attn_kernel<128, false>, AttnCfg<128>::THREADS, AttnCfg<128>::SMEM_BYTES);
   else
@@ -692,6 +705,53 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
   if (o == k || o == v) return SVG_ERR_INVALID_ARG;
   return sparse_attn_impl(qp, k, v, perm_k, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols,
                           scale, perm_q, o, lse, ws, ws_bytes, stream);
+}
+
+svg_status svg_quantize_e4m3(const void *x, int BH, int N, int D, int per_row, void *x8, float *scales,
+                             svg_stream_t stream) {
+  if (!x || !x8 || !scales || !sizes_ok(BH, N) || (per_row != 0 && per_row != 1)) return SVG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(x8, 16) || !aligned(scales, 4) || x == x8) return SVG_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  uint8_t *q = static_cast<uint8_t *>(x8);
+  if (per_row) {
+    const size_t rows = static_cast<size_t>(BH) * N;
+    const size_t per_block = 8 * (256 / D) * 2;   // 8 warps x rows per warp pass x passes per iteration
+    const size_t want = (rows + per_block - 1) / per_block;
+    const int grid = static_cast<int>(want < static_cast<size_t>(num_sms()) * 8 ? want : num_sms() * 8);
+    if (D == 128)
+      quant_rows_e4m3_kernel<128><<<grid, 256, 0, s>>>(xb, rows, q, scales);
+    else
+      quant_rows_e4m3_kernel<64><<<grid, 256, 0, s>>>(xb, rows, q, scales);
+    return launch_status("quant_rows_e4m3_kernel");
+  }
+  // per head: amax (float bits, max-folded into the zeroed scales), quantise, amax -> scale
+  const size_t per_head = static_cast<size_t>(N) * D;
+  int chunks = static_cast<int>((per_head / 8 + 255) / 256);
+  const int cap = (num_sms() * 8 + BH - 1) / BH;
+  if (chunks > cap) chunks = cap;
+  if (chunks < 1) chunks = 1;
+  int32_t *bits = reinterpret_cast<int32_t *>(scales);
+  svg_status st = cuda_status(cudaMemsetAsync(bits, 0, static_cast<size_t>(BH) * sizeof(int32_t), s),
+                              "cudaMemsetAsync(scales)");
+  if (st != SVG_OK) return st;
+  head_amax_kernel<<<dim3(chunks, BH), 256, 0, s>>>(xb, per_head, bits);
+  if ((st = launch_status("head_amax_kernel")) != SVG_OK) return st;
+  quant_heads_e4m3_kernel<<<dim3(chunks, BH), 256, 0, s>>>(xb, per_head, bits, q);
+  if ((st = launch_status("quant_heads_e4m3_kernel")) != SVG_OK) return st;
+  head_scale_kernel<<<(BH + 255) / 256, 256, 0, s>>>(bits, BH);
+  return launch_status("head_scale_kernel");
+}
+
+svg_status svg_sparse_attn_fp8(const void *q8, const float *q_scale, const void *k8, const float *k_scale,
+                               const void *vp, int BH, int N, int D, const int32_t *q_off, int Cq,
+                               const int32_t *k_off, int Ck, const int32_t *sel_count, const int32_t *sel_cols,
+                               float scale, const int32_t *perm_q, void *o, float *lse, void *ws,
+                               size_t ws_bytes, svg_stream_t stream) {
+  if (!q_scale || !k_scale) return SVG_ERR_INVALID_ARG;
+  return sparse_attn_impl(q8, k8, vp, nullptr, BH, N, D, q_off, Cq, k_off, Ck, sel_count, sel_cols, scale,
+                          perm_q, o, lse, ws, ws_bytes, stream, q_scale, k_scale);
 }
 
 }  // extern "C"
