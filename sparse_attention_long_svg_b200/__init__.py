@@ -8,7 +8,9 @@ library and a CUDA device and raises otherwise.
 
 Stages (Sparse VideoGen2, section 2): ``kmeans`` -> ``permute`` ->
 ``select_topp`` -> ``sparse_attn`` -> ``unpermute``; ``svg_attention`` runs
-the whole layer.
+the whole layer.  Options: ``sparse_attn_gather`` (K/V rows fetched through
+the K permutation), ``dynrad_select`` (DynamicRad block masks),
+``quantize_e4m3`` + ``sparse_attn_fp8`` (Q K^T on 8-bit tensor cores).
 """
 from __future__ import annotations
 
