@@ -237,8 +237,9 @@ def kernel_launches_per_step(iters: int, qk_fp8: bool = False) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
     per_kmeans = 1 + 4 * iters               # split + T x (assign, refine, bucket, accumulate); ||x||^2 in the first assign
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
-    quant = (1 + 3) if qk_fp8 else 0         # Q per row; K per head: amax, quantise, scale
-    return 2 * per_kmeans + 2 * per_permute + 1 + quant + 4   # select; [quantise]; plan x3 + attention
+    if qk_fp8:   # Q's permutation moves no rows; quantise Q per row, K per head (amax, quantise, scale)
+        return 2 * per_kmeans + 2 * per_permute - 1 + 1 + 4 + 4
+    return 2 * per_kmeans + 2 * per_permute + 1 + 4       # select; plan x3 + attention (un-permute fused)
 
 
 def attention_pairs(layer, wl):
@@ -320,12 +321,16 @@ def run_svg(args, wl):
         svg.kmeans(k, mu_k, T, layer.assign_k, layer.n_k, layer.workspace)
         if ev:
             ev[2].record()
-        svg.permute(layer.assign_q, wl.cq, [q], [layer.qp], layer.perm_q, layer.q_off, layer.workspace)
-        if args.kv_gather:       # K permutation only: attention fetches K/V rows through it
-            svg.permute(layer.assign_k, wl.ck, [], [], layer.perm_k, layer.k_off, layer.workspace)
+        if args.qk_fp8:          # Q and K are gathered by their quantisation; only V is moved
+            svg.permute(layer.assign_q, wl.cq, [], [], layer.perm_q, layer.q_off, layer.workspace)
+            svg.permute(layer.assign_k, wl.ck, [v], [layer.vp], layer.perm_k, layer.k_off, layer.workspace)
         else:
-            svg.permute(layer.assign_k, wl.ck, [k, v], [layer.kp, layer.vp], layer.perm_k, layer.k_off,
-                        layer.workspace)
+            svg.permute(layer.assign_q, wl.cq, [q], [layer.qp], layer.perm_q, layer.q_off, layer.workspace)
+            if args.kv_gather:   # K permutation only: attention fetches K/V rows through it
+                svg.permute(layer.assign_k, wl.ck, [], [], layer.perm_k, layer.k_off, layer.workspace)
+            else:
+                svg.permute(layer.assign_k, wl.ck, [k, v], [layer.kp, layer.vp], layer.perm_k, layer.k_off,
+                            layer.workspace)
         if ev:
             ev[3].record()
         svg.select_topp(mu_q, layer.n_q, mu_k, layer.n_k, p, 0.0, layer.sel_count, layer.sel_cols)
@@ -334,9 +339,9 @@ def run_svg(args, wl):
         if args.kv_gather:
             svg.sparse_attn_gather(layer.qp, k, v, layer.perm_k, layer.q_off, layer.k_off, layer.sel_count,
                                    layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
-        elif args.qk_fp8:        # E4M3 Q (per row) and K (per head), then attention with 8-bit Q K^T
-            svg.quantize_e4m3(layer.qp, True, q8, sq)
-            svg.quantize_e4m3(layer.kp, False, k8, sk)
+        elif args.qk_fp8:        # E4M3 Q (per row) and K (per head) gathered by the permutations, then attention
+            svg.quantize_e4m3(q, True, q8, sq, perm=layer.perm_q)
+            svg.quantize_e4m3(k, False, k8, sk, perm=layer.perm_k)
             svg.sparse_attn_fp8(q8, sq, k8, sk, layer.vp, layer.q_off, layer.k_off, layer.sel_count,
                                 layer.sel_cols, 0.0, out, workspace=layer.workspace, perm_q=layer.perm_q)
         else:
@@ -530,7 +535,8 @@ def run_svg(args, wl):
             "config": dict(workload_config(wl, world, BH, T, p),
                            kv=("gathered by the attention kernel through the K permutation" if args.kv_gather
                                else "permuted copies written by svg_permute"),
-                           **({"qk": "E4M3 Q (per-row scales) and K (per-head scales), quantised each step"}
+                           **({"qk": "E4M3 Q (per-row scales) and K (per-head scales), quantised each step while "
+                                     "gathered into permuted order"}
                               if args.qk_fp8 else {})),
             "attn_ms": stage_ms["attn+unpermute"], "attn_eff_tflops": attn_tflops,
             "attn_frac_of_bf16_peak": attn_tflops / tc_peak, "density": density, "stages": stages,

@@ -224,6 +224,11 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
  *   per_row = 0   one scale per head over all N*D values, scales [BH]  (for K)
  * D = 64 or 128.  x and x8 16-byte aligned, not aliased.  The per-head form
  * zeroes `scales` (stream-ordered) before reducing into it.
+ * perm [BH, N] int32 is optional: with it the rows are gathered on the way,
+ * x8[h][i] = E4M3(x[h][perm[h][i]] / s) (per-row scales follow the output
+ * row; a head's scale does not depend on the order), so the permuted Q and K
+ * of svg_permute need not be written in bf16 first.  A perm entry outside
+ * [0, N) gives a zero row and is flagged with SVG_ERR_DEVICE_CHECK.
  *
  * svg_sparse_attn_fp8: svg_sparse_attn / svg_sparse_attn_unpermuted with
  * q8 [BH, N, D] and k8 [BH, N, D] E4M3 (permuted, as svg_quantize_e4m3 makes
@@ -233,8 +238,8 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
  * workspace is svg_sparse_attn_workspace_size(BH, N, Cq) bytes; other
  * arguments and the error behaviour are those of svg_sparse_attn.
  */
-svg_status svg_quantize_e4m3(const void *x, int BH, int N, int D, int per_row, void *x8, float *scales,
-                             svg_stream_t stream);
+svg_status svg_quantize_e4m3(const void *x, const int32_t *perm, int BH, int N, int D, int per_row, void *x8,
+                             float *scales, svg_stream_t stream);
 svg_status svg_sparse_attn_fp8(const void *q8, const float *q_scale, const void *k8, const float *k_scale,
                                const void *vp, int BH, int N, int D, const int32_t *q_off, int Cq,
                                const int32_t *k_off, int Ck, const int32_t *sel_count, const int32_t *sel_cols,

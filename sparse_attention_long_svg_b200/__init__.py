@@ -53,7 +53,7 @@ SIGNATURES = {
     "svg_sparse_attn_gather": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P,
                                     _SZ, _P]),
     "svg_unpermute": (_I, [_P, _P, _I, _I, _I, _P, _P]),
-    "svg_quantize_e4m3": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "svg_quantize_e4m3": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "svg_sparse_attn_fp8": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _F, _P, _P, _P, _P, _SZ,
                                  _P]),
     "svg_dynrad_num_blocks": (_I, [_I, _I, _I]),
@@ -313,19 +313,22 @@ def sparse_attn_gather(qp, k, v, perm_k, q_off, k_off, sel_count, sel_cols, scal
     return op, lse
 
 
-def quantize_e4m3(x, per_row: bool, x8=None, scales=None, stream=None):
+def quantize_e4m3(x, per_row: bool, x8=None, scales=None, stream=None, perm=None):
     """E4M3 copy of x [BH, N, D] bf16 and its float32 scales (svg_quantize_e4m3):
     per_row -> scales [BH, N] (one per row, for Q), else [BH] (one per head, for K).
-    Returns (x8 as torch.float8_e4m3fn, scales)."""
+    With ``perm`` [BH, N] int32 the rows are gathered on the way: row i of head h
+    is quantised from row perm[h, i].  Returns (x8 as torch.float8_e4m3fn, scales)."""
     lib = load_library()
     _need(x, "x", torch.bfloat16, 3)
+    if perm is not None:
+        _need(perm, "perm", torch.int32, 2)
     BH, N, D = x.shape
     if x8 is None:
         x8 = torch.empty((BH, N, D), dtype=torch.float8_e4m3fn, device=x.device)
     if scales is None:
         scales = torch.empty((BH, N) if per_row else (BH,), dtype=torch.float32, device=x.device)
-    _check("svg_quantize_e4m3", lib.svg_quantize_e4m3(_ptr(x), BH, N, D, 1 if per_row else 0, _ptr(x8),
-                                                      _ptr(scales), _stream(stream)))
+    _check("svg_quantize_e4m3", lib.svg_quantize_e4m3(_ptr(x), _ptr(perm), BH, N, D, 1 if per_row else 0,
+                                                      _ptr(x8), _ptr(scales), _stream(stream)))
     return x8, scales
 
 
@@ -458,9 +461,9 @@ class LayerState:
     k_off: torch.Tensor
     sel_count: torch.Tensor
     sel_cols: torch.Tensor
-    qp: torch.Tensor
-    kp: Optional[torch.Tensor]     # permuted K and V; None when attention gathered rows through perm_k
-    vp: Optional[torch.Tensor]
+    qp: Optional[torch.Tensor]     # permuted Q; None with qk_fp8 (Q quantised while gathered)
+    kp: Optional[torch.Tensor]     # permuted K; None with kv_gather (rows fetched through perm_k) or qk_fp8
+    vp: Optional[torch.Tensor]     # permuted V; None with kv_gather
     op: Optional[torch.Tensor]     # permuted output; None when the un-permutation was fused
 
 
@@ -498,20 +501,26 @@ class SvgLayer:
         (no permuted output copy, ``LayerState.op`` is None), else attention + svg_unpermute.
         With ``kv_gather`` K and V are not permuted: the attention kernel fetches their rows
         through the K permutation (``LayerState.kp``/``vp`` are None); requires fused_unpermute.
-        With ``qk_fp8`` the permuted Q and K are quantised to E4M3 (per-row / per-head scales)
+        With ``qk_fp8`` Q and K are quantised to E4M3 (per-row / per-head scales) while they are
+        gathered into permuted order (no bf16 permuted copies: ``LayerState.qp``/``kp`` are None)
         and S = Q K^T runs on 8-bit operands; D must be 128."""
         if qk_fp8 and kv_gather:
             raise ValueError("qk_fp8 and kv_gather cannot be combined")
         kmeans(q, mu_q, iters, self.assign_q, self.n_q, self.workspace, stream)
         kmeans(k, mu_k, iters, self.assign_k, self.n_k, self.workspace, stream)
         Cq, Ck = mu_q.shape[1], mu_k.shape[1]
-        permute(self.assign_q, Cq, [q], [self.qp], self.perm_q, self.q_off, self.workspace, stream)
-        if kv_gather:
-            if not fused_unpermute:
-                raise ValueError("kv_gather requires fused_unpermute")
-            permute(self.assign_k, Ck, [], [], self.perm_k, self.k_off, self.workspace, stream)
+        if qk_fp8:     # Q and K are gathered by the quantisation below; only V is moved here
+            permute(self.assign_q, Cq, [], [], self.perm_q, self.q_off, self.workspace, stream)
+            permute(self.assign_k, Ck, [v], [self.vp], self.perm_k, self.k_off, self.workspace, stream)
         else:
-            permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace, stream)
+            permute(self.assign_q, Cq, [q], [self.qp], self.perm_q, self.q_off, self.workspace, stream)
+            if kv_gather:
+                if not fused_unpermute:
+                    raise ValueError("kv_gather requires fused_unpermute")
+                permute(self.assign_k, Ck, [], [], self.perm_k, self.k_off, self.workspace, stream)
+            else:
+                permute(self.assign_k, Ck, [k, v], [self.kp, self.vp], self.perm_k, self.k_off, self.workspace,
+                        stream)
         select_topp(mu_q, self.n_q, mu_k, self.n_k, p, scale, self.sel_count, self.sel_cols, stream)
         if kv_gather:
             if out is None:
@@ -530,8 +539,8 @@ class SvgLayer:
                 self.fp8 = (torch.empty((BH, N, D), **f8), torch.empty((BH, N), **f32),
                             torch.empty((BH, N, D), **f8), torch.empty((BH,), **f32))
             q8, sq, k8, sk = self.fp8
-            quantize_e4m3(self.qp, True, q8, sq, stream)
-            quantize_e4m3(self.kp, False, k8, sk, stream)
+            quantize_e4m3(q, True, q8, sq, stream, perm=self.perm_q)
+            quantize_e4m3(k, False, k8, sk, stream, perm=self.perm_k)
             if fused_unpermute:
                 if out is None:
                     out = torch.empty_like(q)
@@ -543,7 +552,10 @@ class SvgLayer:
                                 scale, self.op, workspace=self.workspace, stream=stream)
                 out = unpermute(self.op, self.perm_q, out, stream)
                 op = self.op
-        elif fused_unpermute:
+            return out, LayerState(mu_q, mu_k, self.assign_q, self.assign_k, self.n_q, self.n_k, self.perm_q,
+                                   self.perm_k, self.q_off, self.k_off, self.sel_count, self.sel_cols, None, None,
+                                   self.vp, op)
+        if fused_unpermute:
             if out is None:
                 out = torch.empty_like(q)
             sparse_attn(self.qp, self.kp, self.vp, self.q_off, self.k_off, self.sel_count, self.sel_cols, scale,

@@ -26,26 +26,48 @@ __device__ __forceinline__ uint32_t e4m3_byte(float v, float s) {
   return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Per-row scales: each lane converts 8 consecutive channels (one 16-byte
-// load); the D / 8 lanes of a row reduce its amax with shuffles, so a warp
-// covers 256 / D rows per pass, and two passes are in flight per iteration.
-template <int D>
-__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const __nv_bfloat16 *__restrict__ x, size_t rows,
-                                                              uint8_t *__restrict__ x8, float *__restrict__ scales) {
+// Source row of output row r (r = h * N + i): row i itself, or row perm[r] of
+// the same head (gathered); -1 for a permutation entry outside [0, N), which
+// is recorded and quantised as a zero row.
+__device__ __forceinline__ long long quant_src_row(const int32_t *perm, size_t r, int N) {
+  if (perm == nullptr) return static_cast<long long>(r);
+  const int t = __ldg(perm + r);
+  if (t < 0 || t >= N) {
+    record_error(SVG_ERR_DEVICE_CHECK, SITE_PERMUTE_RANGE);
+    return -1;
+  }
+  return static_cast<long long>(r - r % static_cast<size_t>(N)) + t;
+}
+
+// Quantisation of rows: each lane converts 8 consecutive channels (one
+// 16-byte load), D / 8 lanes a row, so a warp covers 256 / D rows per pass
+// and U passes are in flight per iteration.  PER_ROW: the row's amax (by
+// shuffles) gives its scale, written to scales[r]; otherwise the head's amax
+// is read from amax_bits[r / N].  With perm the source row is gathered.
+template <int D, bool PER_ROW>
+__global__ void __launch_bounds__(256) quant_e4m3_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                         const int32_t *__restrict__ perm, int N, size_t rows,
+                                                         const int32_t *__restrict__ amax_bits,
+                                                         uint8_t *__restrict__ x8, float *__restrict__ scales) {
   constexpr int LPR = D / 8;           // lanes per row
   constexpr int RPW = 32 / LPR;        // rows per warp pass
-  constexpr int U = 2;                 // passes per iteration
+  constexpr int U = 4;                 // passes per iteration
   const int lane = threadIdx.x & 31;
   const int sub = lane / LPR, c = lane % LPR;
   const size_t warp = static_cast<size_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const size_t warps = static_cast<size_t>(gridDim.x) * (blockDim.x >> 5);
   for (size_t r0 = warp * (RPW * U); r0 < rows; r0 += warps * (RPW * U)) {
-    uint4 u[U];
+    long long src[U];
 #pragma unroll
     for (int i = 0; i < U; ++i) {
       const size_t r = r0 + i * RPW + sub;
-      u[i] = r < rows ? __ldcs(reinterpret_cast<const uint4 *>(x + r * D) + c) : make_uint4(0, 0, 0, 0);
+      src[i] = r < rows ? quant_src_row(perm, r, N) : -1;
     }
+    uint4 u[U];
+#pragma unroll
+    for (int i = 0; i < U; ++i)
+      u[i] = src[i] >= 0 ? __ldcs(reinterpret_cast<const uint4 *>(x + static_cast<size_t>(src[i]) * D) + c)
+                         : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int i = 0; i < U; ++i) {
       const size_t r = r0 + i * RPW + sub;
@@ -57,12 +79,17 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const __nv_bfloat1
         v[2 * j] = __low2float(b);
         v[2 * j + 1] = __high2float(b);
       }
-      float m = 0.f;
+      float s;
+      if constexpr (PER_ROW) {
+        float m = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float s = e4m3_scale(m);
+        for (int o = LPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        s = e4m3_scale(m);
+      } else {
+        s = e4m3_scale(__int_as_float(__ldg(amax_bits + (r < rows ? r / N : 0))));
+      }
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -71,7 +98,7 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const __nv_bfloat1
       }
       if (r < rows) {
         reinterpret_cast<uint2 *>(x8 + r * D)[c] = make_uint2(lo, hi);
-        if (c == 0) scales[r] = s;
+        if (PER_ROW && c == 0) scales[r] = s;
       }
     }
   }
@@ -113,38 +140,6 @@ __global__ void __launch_bounds__(256) head_amax_kernel(const __nv_bfloat16 *__r
     float b = 0.f;
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) b = fmaxf(b, wmax[w]);
     atomicMax(amax_bits + h, __float_as_int(b));
-  }
-}
-
-// Quantises each head with the scale of its amax (read from amax_bits).
-__global__ void __launch_bounds__(256) quant_heads_e4m3_kernel(const __nv_bfloat16 *__restrict__ x, size_t per_head,
-                                                               const int32_t *__restrict__ amax_bits,
-                                                               uint8_t *__restrict__ x8) {
-  const int h = blockIdx.y;
-  const float s = e4m3_scale(__int_as_float(amax_bits[h]));
-  const uint4 *src = reinterpret_cast<const uint4 *>(x + static_cast<size_t>(h) * per_head);
-  uint2 *dst = reinterpret_cast<uint2 *>(x8 + static_cast<size_t>(h) * per_head);
-  const size_t groups = per_head / 8;
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  for (size_t g0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; g0 < groups; g0 += 2 * stride) {
-    uint4 u[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const size_t g = g0 + k * stride;
-      u[k] = g < groups ? __ldcs(src + g) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-      uint32_t out[2] = {0, 0};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
-        out[i >> 1] |= (e4m3_byte(__low2float(b), s) | (e4m3_byte(__high2float(b), s) << 8)) << (16 * (i & 1));
-      }
-      const size_t g = g0 + k * stride;
-      if (g < groups) dst[g] = make_uint2(out[0], out[1]);
-    }
   }
 }
 

@@ -707,24 +707,24 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
                           scale, perm_q, o, lse, ws, ws_bytes, stream);
 }
 
-svg_status svg_quantize_e4m3(const void *x, int BH, int N, int D, int per_row, void *x8, float *scales,
-                             svg_stream_t stream) {
+svg_status svg_quantize_e4m3(const void *x, const int32_t *perm, int BH, int N, int D, int per_row, void *x8,
+                             float *scales, svg_stream_t stream) {
   if (!x || !x8 || !scales || !sizes_ok(BH, N) || (per_row != 0 && per_row != 1)) return SVG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SVG_ERR_UNSUPPORTED;
   if (!aligned(x, 16) || !aligned(x8, 16) || !aligned(scales, 4) || x == x8) return SVG_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   uint8_t *q = static_cast<uint8_t *>(x8);
+  const size_t rows = static_cast<size_t>(BH) * N;
+  const size_t per_block = 8 * (256 / D) * 4;   // 8 warps x rows per warp pass x passes per iteration
+  const size_t want = (rows + per_block - 1) / per_block;
+  const int grid = static_cast<int>(want < static_cast<size_t>(num_sms()) * 8 ? want : num_sms() * 8);
   if (per_row) {
-    const size_t rows = static_cast<size_t>(BH) * N;
-    const size_t per_block = 8 * (256 / D) * 2;   // 8 warps x rows per warp pass x passes per iteration
-    const size_t want = (rows + per_block - 1) / per_block;
-    const int grid = static_cast<int>(want < static_cast<size_t>(num_sms()) * 8 ? want : num_sms() * 8);
     if (D == 128)
-      quant_rows_e4m3_kernel<128><<<grid, 256, 0, s>>>(xb, rows, q, scales);
+      quant_e4m3_kernel<128, true><<<grid, 256, 0, s>>>(xb, perm, N, rows, nullptr, q, scales);
     else
-      quant_rows_e4m3_kernel<64><<<grid, 256, 0, s>>>(xb, rows, q, scales);
-    return launch_status("quant_rows_e4m3_kernel");
+      quant_e4m3_kernel<64, true><<<grid, 256, 0, s>>>(xb, perm, N, rows, nullptr, q, scales);
+    return launch_status("quant_e4m3_kernel");
   }
   // per head: amax (float bits, max-folded into the zeroed scales), quantise, amax -> scale
   const size_t per_head = static_cast<size_t>(N) * D;
@@ -738,8 +738,11 @@ svg_status svg_quantize_e4m3(const void *x, int BH, int N, int D, int per_row, v
   if (st != SVG_OK) return st;
   head_amax_kernel<<<dim3(chunks, BH), 256, 0, s>>>(xb, per_head, bits);
   if ((st = launch_status("head_amax_kernel")) != SVG_OK) return st;
-  quant_heads_e4m3_kernel<<<dim3(chunks, BH), 256, 0, s>>>(xb, per_head, bits, q);
-  if ((st = launch_status("quant_heads_e4m3_kernel")) != SVG_OK) return st;
+  if (D == 128)
+    quant_e4m3_kernel<128, false><<<grid, 256, 0, s>>>(xb, perm, N, rows, bits, q, nullptr);
+  else
+    quant_e4m3_kernel<64, false><<<grid, 256, 0, s>>>(xb, perm, N, rows, bits, q, nullptr);
+  if ((st = launch_status("quant_e4m3_kernel")) != SVG_OK) return st;
   head_scale_kernel<<<(BH + 255) / 256, 256, 0, s>>>(bits, BH);
   return launch_status("head_scale_kernel");
 }

@@ -123,11 +123,11 @@ def test_invalid_arguments_are_rejected_before_launch(lib):
     assert dyn(f, 30, 96, 3, 4, 2) == 2
     assert dyn(f, 30, 64, 3, 4, 2, ws=8) == 3
     # E4M3 quantisation: unsupported D, per_row not 0/1, x8 aliasing x, null scales, misaligned x
-    assert lib.svg_quantize_e4m3(f, 1, 16, 96, 1, g, f, nul) == 2
-    assert lib.svg_quantize_e4m3(f, 1, 16, 64, 2, g, f, nul) == 1
-    assert lib.svg_quantize_e4m3(f, 1, 16, 64, 1, f, g, nul) == 1
-    assert lib.svg_quantize_e4m3(f, 1, 16, 64, 0, g, nul, nul) == 1
-    assert lib.svg_quantize_e4m3(_p(FAKE + 2), 1, 16, 64, 0, g, f, nul) == 1
+    assert lib.svg_quantize_e4m3(f, nul, 1, 16, 96, 1, g, f, nul) == 2
+    assert lib.svg_quantize_e4m3(f, nul, 1, 16, 64, 2, g, f, nul) == 1
+    assert lib.svg_quantize_e4m3(f, nul, 1, 16, 64, 1, f, g, nul) == 1
+    assert lib.svg_quantize_e4m3(f, nul, 1, 16, 64, 0, g, nul, nul) == 1
+    assert lib.svg_quantize_e4m3(_p(FAKE + 2), nul, 1, 16, 64, 0, g, f, nul) == 1
     # 8-bit Q K^T attention: missing scales, D other than 128, small workspace
     fp8 = lambda qs, ks, N, D, ws: lib.svg_sparse_attn_fp8(f, qs, f, ks, f, 1, N, D, f, 2, f, 2, f, f, 0.0, nul,
                                                            g, nul, f, ws, nul)

@@ -23,6 +23,7 @@ def test_launch_count_per_step():
     # select; two planning kernels + attention (un-permute fused)
     assert bench.kernel_launches_per_step(5) == 2 * (1 + 4 * 5) + 2 * 4 + 1 + 4 == 55
     assert bench.kernel_launches_per_step(2) == 2 * (1 + 4 * 2) + 13
+    assert bench.kernel_launches_per_step(5, qk_fp8=True) == 55 - 1 + 4 == 58
 
 
 def test_workload_config_keys():

@@ -91,16 +91,41 @@ def test_quantize_heads_bit_exact(D):
         assert np.array_equal(got8[h], want8), (h, np.argwhere(got8[h] != want8)[:5])
 
 
+@pytest.mark.parametrize("per_row", [True, False])
+def test_quantize_gathered_equals_quantize_of_gathered_rows(per_row):
+    """Quantising through a permutation equals gathering the rows first, bit for bit;
+    a permutation entry out of range gives a zero row and the device check."""
+    BH, N, D = 3, 517, 128
+    x = awkward_rows(BH * N, D, seed=7).reshape(BH, N, D)
+    rng = np.random.default_rng(8)
+    perm = np.stack([rng.permutation(N) for _ in range(BH)]).astype(np.int32)
+    xg = np.stack([x[h][perm[h]] for h in range(BH)])
+    dx, dp = dev_bf16(x), dev_i32(perm)
+    a8, sa = svg.quantize_e4m3(dx, per_row=per_row, perm=dp)
+    b8, sb = svg.quantize_e4m3(dev_bf16(xg), per_row=per_row)
+    torch.cuda.synchronize()
+    assert svg.get_error() == 0
+    assert torch.equal(a8.view(torch.uint8), b8.view(torch.uint8)) and torch.equal(sa, sb)
+    bad = perm.copy()
+    bad[1, 5] = N + 3
+    c8, sc = svg.quantize_e4m3(dx, per_row=per_row, perm=dev_i32(bad))
+    torch.cuda.synchronize()
+    assert svg.get_error() == 6                  # SVG_ERR_DEVICE_CHECK
+    assert torch.count_nonzero(c8[1, 5].view(torch.uint8)).item() == 0
+    if per_row:
+        assert sc[1, 5].item() == 1.0
+
+
 def test_quantize_rejects_bad_arguments():
     lib = svg.load_library()
     x = torch.zeros((2, 8, 128), dtype=torch.bfloat16, device="cuda")
     x8 = torch.empty((2, 8, 128), dtype=torch.uint8, device="cuda")
     s = torch.empty(16, dtype=torch.float32, device="cuda")
     P = svg._ptr
-    assert lib.svg_quantize_e4m3(P(x), 2, 8, 96, 1, P(x8), P(s), None) == 2        # D unsupported
-    assert lib.svg_quantize_e4m3(P(x), 2, 8, 128, 2, P(x8), P(s), None) == 1       # per_row not 0/1
-    assert lib.svg_quantize_e4m3(P(x), 2, 8, 128, 1, P(x), P(s), None) == 1        # x8 aliases x
-    assert lib.svg_quantize_e4m3(None, 2, 8, 128, 1, P(x8), P(s), None) == 1
+    assert lib.svg_quantize_e4m3(P(x), None, 2, 8, 96, 1, P(x8), P(s), None) == 2        # D unsupported
+    assert lib.svg_quantize_e4m3(P(x), None, 2, 8, 128, 2, P(x8), P(s), None) == 1       # per_row not 0/1
+    assert lib.svg_quantize_e4m3(P(x), None, 2, 8, 128, 1, P(x), P(s), None) == 1        # x8 aliases x
+    assert lib.svg_quantize_e4m3(None, None, 2, 8, 128, 1, P(x8), P(s), None) == 1
 
 
 CASES = {
@@ -216,8 +241,9 @@ def test_fp8_layer_equals_stages_and_graph(case_data):
     out = out.clone()
     torch.cuda.synchronize()
     assert svg.get_error() == 0
-    q8, sq = svg.quantize_e4m3(st.qp, per_row=True)
-    k8, sk = svg.quantize_e4m3(st.kp, per_row=False)
+    assert st.qp is None and st.kp is None      # Q and K were quantised while gathered
+    q8, sq = svg.quantize_e4m3(q, per_row=True, perm=st.perm_q)
+    k8, sk = svg.quantize_e4m3(k, per_row=False, perm=st.perm_k)
     want, _ = svg.sparse_attn_fp8(q8, sq, k8, sk, st.vp, st.q_off, st.k_off, st.sel_count, st.sel_cols,
                                   perm_q=st.perm_q)
     torch.cuda.synchronize()
@@ -255,3 +281,24 @@ def test_fp8_full_size_480p():
                                         1.0 / math.sqrt(D), rows=prow)
         have = got[h][torch.from_numpy(perm_q[h][prow]).to(got.device)].cpu().numpy()
         check_attention(have, op[prow], f"480p fp8 head {h}")
+
+
+def test_fp8_degenerate_inputs(case_data):
+    """Degenerate inputs against the oracle: a head whose K is all zero (scale 1, every
+    logit 0: uniform weights over the selected keys), zero query rows, and Q and K scaled
+    by 8 (logits up to ~10^3 in magnitude: the softmax's running max must hold)."""
+    L, ref = case_data("small-d128")
+    qp, kp, vp, q_off, k_off, cnt, cols = permuted_inputs(L, ref)
+    qp, kp = qp.copy(), kp.copy()
+    kp[0] = 0.0                                  # head 0: K all zero
+    qp[1, ::7] = 0.0                             # head 1: every 7th query row zero
+    qp[2] = synth.round_bf16(qp[2] * 8.0)        # head 2: logits x 64
+    kp[2] = synth.round_bf16(kp[2] * 8.0)
+    op, lse = run_fp8(qp, kp, vp, q_off, k_off, cnt, cols)
+    got, got_lse = host_f32(op), lse.cpu().numpy()
+    D = qp.shape[2]
+    for h in range(qp.shape[0]):
+        sel = [s.cols for s in ref[h].selection]
+        want, want_lse = f8.sparse_attention_fp8(qp[h], kp[h], vp[h], q_off[h], k_off[h], sel, 1.0 / math.sqrt(D))
+        check_attention(got[h], want, f"degenerate head {h}")
+        assert np.max(np.abs(got_lse[h] - want_lse) / np.maximum(1.0, np.abs(want_lse))) < 1e-3
