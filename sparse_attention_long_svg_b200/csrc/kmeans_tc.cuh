@@ -350,6 +350,8 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
       const int h = u / tiles, n0 = (u % tiles) * Cfg::BM;
       const bool valid = n0 + row < N;
       const float *nh = norms + static_cast<size_t>(h) * Cpad;
+      // ||x||^2 of later rounds is read now: the load completes while the chunks are reduced
+      const float xx_ld = !make_xnorm && valid ? __ldg(xnorm + static_cast<size_t>(h) * N + n0 + row) : 0.f;
       float best = kBig, second = kBig;
       int arg = 0x7fffffff, arg2 = -1;
       float xx = 0.f;   // ||x||^2 of this row (first round: from the x tile in shared memory)
@@ -468,7 +470,7 @@ __global__ void __launch_bounds__(KmCfg<D, SINGLE>::THREADS, 1)
       if (valid && !live) record_error(SVG_ERR_DEVICE_CHECK, SITE_KMEANS_RANGE);
       bool tie = false;
       if (live && arg2 >= 0 && arg2 < C) {
-        if (!make_xnorm) xx = xnorm[static_cast<size_t>(h) * N + n0 + row];
+        if (!make_xnorm) xx = xx_ld;
         const float mm = fmaxf(__ldg(nh + arg), __ldg(nh + arg2));
         tie = second - best <= 0x1p-14f * (fabsf(best) + fabsf(second) + xx + mm);
       }
