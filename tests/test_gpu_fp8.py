@@ -302,3 +302,39 @@ def test_fp8_degenerate_inputs(case_data):
         want, want_lse = f8.sparse_attention_fp8(qp[h], kp[h], vp[h], q_off[h], k_off[h], sel, 1.0 / math.sqrt(D))
         check_attention(got[h], want, f"degenerate head {h}")
         assert np.max(np.abs(got_lse[h] - want_lse) / np.maximum(1.0, np.abs(want_lse))) < 1e-3
+
+
+def rand_bf16(shape, seed):
+    return synth.round_bf16(np.random.default_rng(seed).standard_normal(shape).astype(np.float32))
+
+
+@pytest.mark.parametrize("case", ["max-clusters", "one-token-clusters", "empty-clusters"])
+def test_fp8_layer_edge_cases(case):
+    """The 8-bit layer on the edge cases of the bf16 path, every row against the oracle on the
+    GPU's clustering and selection: 1024 clusters with a ragged N = 4100 (max k-clusters per row,
+    a partial last tile), one token per cluster (C = N), duplicated seeds (empty clusters) with p = 0.01."""
+    if case == "max-clusters":
+        q, k, v = (rand_bf16((1, 4100, 128), s) for s in (20, 21, 22))
+        mu_q0, mu_k0, iters, p = q[:, :1024], k[:, :1024], 1, 0.9
+    elif case == "one-token-clusters":
+        q, k, v = (rand_bf16((1, 96, 128), s) for s in (23, 24, 25))
+        mu_q0, mu_k0, iters, p = q.copy(), k.copy(), 2, 0.7
+    else:
+        q, k, v = (rand_bf16((2, 1500, 128), s) for s in (26, 27, 28))
+        mu_q0, mu_k0, iters, p = np.repeat(q[:, :5], 4, axis=1), np.repeat(k[:, :9], 3, axis=1), 3, 0.01
+    H, N, D = q.shape
+    layer = svg.SvgLayer(H, N, D, mu_q0.shape[1], mu_k0.shape[1])
+    out, st = layer(dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_f32(mu_q0), dev_f32(mu_k0), iters, p, qk_fp8=True)
+    torch.cuda.synchronize()
+    assert svg.get_error() == 0
+    got = host_f32(out)
+    sel = selection_lists(st.sel_count, st.sel_cols)
+    for h in range(H):
+        perm_q, perm_k = st.perm_q.cpu().numpy()[h], st.perm_k.cpu().numpy()[h]
+        op, _ = f8.sparse_attention_fp8(so.gather_rows(q[h], perm_q), so.gather_rows(k[h], perm_k),
+                                        so.gather_rows(v[h], perm_k), st.q_off.cpu().numpy()[h],
+                                        st.k_off.cpu().numpy()[h], sel[h], 1.0 / math.sqrt(D))
+        check_attention(got[h], so.scatter_rows(op, perm_q), f"fp8 {case} head {h}")
+    if case == "empty-clusters":
+        n_q, cnt = st.n_q.cpu().numpy(), st.sel_count.cpu().numpy()
+        assert (n_q == 0).any() and np.all(cnt[n_q == 0] == 0) and np.all(cnt[n_q > 0] >= 1)
