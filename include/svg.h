@@ -231,9 +231,9 @@ svg_status svg_sparse_attn_gather(const void *qp, const void *k, const void *v, 
  * [0, N) gives a zero row and is flagged with SVG_ERR_DEVICE_CHECK.
  *
  * svg_sparse_attn_fp8: svg_sparse_attn / svg_sparse_attn_unpermuted with
- * q8 [BH, N, D] and k8 [BH, N, D] E4M3 (permuted, as svg_quantize_e4m3 makes
- * them from qp and kp), q_scale [BH * N] and k_scale [BH] their scales, vp
- * bf16.  perm_q optional: with it o (and lse) are in token order, else in
+ * q8 [BH, N, D] and k8 [BH, N, D] E4M3 in permuted row order (svg_quantize_e4m3
+ * of q and k through perm_q and perm_k, or of the permuted qp and kp),
+ * q_scale [BH * N] and k_scale [BH] their scales, vp bf16.  perm_q optional: with it o (and lse) are in token order, else in
  * the Q-permuted order.  D must be 128 (SVG_ERR_UNSUPPORTED otherwise).  The
  * workspace is svg_sparse_attn_workspace_size(BH, N, Cq) bytes; other
  * arguments and the error behaviour are those of svg_sparse_attn.
