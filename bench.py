@@ -257,6 +257,52 @@ def attention_pairs(layer, wl):
     return pairs
 
 
+def pipelined_e2e(host_inputs, out_like, run_step, steps):
+    """End-to-end timing with host buffers: every step copies its inputs from pinned host memory, runs
+    `run_step(device_inputs, device_out, stream)` (which returns the tensor to copy back) and copies the
+    result to pinned host memory, all inside the timed region.  Steps are pipelined over two device
+    buffer sets and three streams: the H2D copies of step i + 1 and the D2H copy of step i - 1 run
+    while step i computes (PCIe is full duplex).  Returns the elapsed milliseconds on this rank."""
+    import torch
+    device = out_like.device
+    hout = [torch.empty(out_like.shape, dtype=out_like.dtype).pin_memory() for _ in range(2)]
+    sets = [([torch.empty(h.shape, dtype=h.dtype, device=device) for h in host_inputs], torch.empty_like(out_like))
+            for _ in range(2)]
+    s_comp = torch.cuda.current_stream()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of set b have landed
+    ev_comp = [torch.cuda.Event() for _ in range(2)]    # step on set b done (inputs free, output ready)
+    ev_d2h = [torch.cuda.Event() for _ in range(2)]     # the output of set b has been copied back
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_comp)
+    s_h2d.wait_event(e0)
+    s_d2h.wait_event(e0)
+    for i in range(steps):
+        b = i % 2
+        dins, dout = sets[b]
+        with torch.cuda.stream(s_h2d):
+            if i >= 2:
+                s_h2d.wait_event(ev_comp[b])            # step i - 2 has consumed this set's inputs
+            for d, h in zip(dins, host_inputs):
+                d.copy_(h, non_blocking=True)
+            ev_in[b].record(s_h2d)
+        s_comp.wait_event(ev_in[b])
+        if i >= 2:
+            s_comp.wait_event(ev_d2h[b])                # step i - 2's output has left this set's buffer
+        o = run_step(dins, dout, s_comp)
+        ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(ev_comp[b])
+            hout[b].copy_(o, non_blocking=True)
+            ev_d2h[b].record(s_d2h)
+    s_comp.wait_stream(s_h2d)
+    s_comp.wait_stream(s_d2h)
+    e1.record(s_comp)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
 def run_svg(args, wl):
     import torch
     rank, world, local = dist_env()
@@ -422,61 +468,22 @@ def run_svg(args, wl):
     all_flops = reduce_sum(flops_layer * args.steps, world, device)
     value = all_flops / (total_ms * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers (pinned), H2D + D2H inside the timed region.
-    # Steps are pipelined over two sets of device buffers and three streams: the H2D copies of step i + 1
-    # and the D2H copy of step i - 1 run while the layer of step i computes (PCIe is full duplex), so the
-    # per-step cost is the slowest of the three rather than their sum.
+    # ---- end to end through the public API with host buffers (pinned), H2D + D2H inside the timed region
     e2e_steps = max(1, min(args.steps, 10))
     hq = torch.from_numpy(synth.bf16_bits(L.q).view(np.int16)).view(torch.bfloat16).pin_memory()
     hk = torch.from_numpy(synth.bf16_bits(L.k).view(np.int16)).view(torch.bfloat16).pin_memory()
     hv = torch.from_numpy(synth.bf16_bits(L.v).view(np.int16)).view(torch.bfloat16).pin_memory()
     hmq, hmk = mu_q0.cpu().pin_memory(), mu_k0.cpu().pin_memory()
-    hout = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    sets = [(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(mu_q0),
-             torch.empty_like(mu_k0), torch.empty_like(q)) for _ in range(2)]
-    s_comp = torch.cuda.current_stream()
-    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of set b have landed
-    ev_comp = [torch.cuda.Event() for _ in range(2)]    # the layer of set b is done (inputs free, output ready)
-    ev_d2h = [torch.cuda.Event() for _ in range(2)]     # the output of set b has been copied back
+
+    def e2e_step(d, o, stream):    # centroids d[3], d[4] are refilled from the host every step
+        return layer(d[0], d[1], d[2], d[3], d[4], T, p, 0.0, o, stream=stream, kv_gather=bool(args.kv_gather),
+                     qk_fp8=bool(args.qk_fp8))[0]
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_comp)
-    s_h2d.wait_event(e0)
-    s_d2h.wait_event(e0)
-    for i in range(e2e_steps):
-        b = i % 2
-        dq, dk, dv, dmq, dmk, dout = sets[b]
-        with torch.cuda.stream(s_h2d):
-            if i >= 2:
-                s_h2d.wait_event(ev_comp[b])            # step i - 2 has consumed this set's inputs
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dmq.copy_(hmq, non_blocking=True)
-            dmk.copy_(hmk, non_blocking=True)
-            ev_in[b].record(s_h2d)
-        s_comp.wait_event(ev_in[b])
-        if i >= 2:
-            s_comp.wait_event(ev_d2h[b])                # step i - 2's output has left this set's buffer
-        o, _ = layer(dq, dk, dv, dmq, dmk, T, p, 0.0, dout, stream=s_comp, kv_gather=bool(args.kv_gather),
-                     qk_fp8=bool(args.qk_fp8))
-        ev_comp[b].record(s_comp)
-        with torch.cuda.stream(s_d2h):
-            s_d2h.wait_event(ev_comp[b])
-            hout[b].copy_(o, non_blocking=True)
-            ev_d2h[b].record(s_d2h)
-    s_comp.wait_stream(s_h2d)
-    s_comp.wait_stream(s_d2h)
-    e1.record(s_comp)
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(e0.elapsed_time(e1), world, device)
+    e2e_ms = reduce_max(pipelined_e2e([hq, hk, hv, hmq, hmk], q, e2e_step, e2e_steps), world, device)
     e2e_value = reduce_sum(flops_layer * e2e_steps, world, device) / (e2e_ms * 1e-3) / 1e12
     h2d = int(3 * hq.numel() * 2 + 2 * hmq.numel() * 4)
-    d2h = int(hout[0].numel() * 2)
-    del sets
+    d2h = int(q.numel() * 2)
 
     # ---- rooflines of the two heavy kernels, from the live event timings.  Each
     # launch is timed on its own (CUDA events around it, inside a timed region of
@@ -699,20 +706,14 @@ def run_dynrad(args, wl):
     e2e_steps = max(1, min(args.steps, 10))
     hq, hk, hv = (torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).pin_memory()
                   for x in (L.q, L.k, L.v))
-    hout = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        step(dq, dk, dv)
-        hout.copy_(out, non_blocking=True)
-    e1.record()
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(e0.elapsed_time(e1), world, device)
+
+    def e2e_step(d, o, stream):
+        with torch.cuda.stream(stream):
+            svg.dynrad_select(d[0], d[1], frames, B, mode, offsets=offs, sel_count=cnt, sel_cols=cols, workspace=ws,
+                              **prm)
+            svg.sparse_attn(d[0], d[1], d[2], offs, offs, cnt, cols, 0.0, o, workspace=ws)
+        return o
+    e2e_ms = reduce_max(pipelined_e2e([hq, hk, hv], q, e2e_step, e2e_steps), world, device)
     e2e_value = reduce_sum(flops_layer * e2e_steps, world, device) / (e2e_ms * 1e-3) / 1e12
 
     tc_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -749,7 +750,9 @@ def run_dynrad(args, wl):
             "stages": {"mask": {"ms": mask_ms}, "attn": {"ms": attn_ms}},
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(3 * hq.numel() * 2),
-                    "d2h_bytes_per_step": int(hout.numel() * 2), "ms_per_step": e2e_ms / e2e_steps},
+                    "d2h_bytes_per_step": int(q.numel() * 2), "ms_per_step": e2e_ms / e2e_steps,
+                    "steps": e2e_steps, "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i "
+                                                      "(two device buffer sets, three streams)"},
             "gpu_launches": (6 if mode == "dynamic" else 5) * args.steps,   # mask (offsets, [means,] select) + plan x3 + attention
             "clocks": clocks.summary(),
         }
