@@ -19,8 +19,7 @@ section 2(a) "Unified candidate set and dual-mode selection":
     a block left empty by the filter keeps its highest-scoring pair.
 
 The page names the hyper-parameters (decay factor gamma, block size B_s,
-thresholds theta) but gives no formulas.  Readings taken (each is listed in
-DESIGN.md):
+thresholds theta) but gives no formulas.  Readings taken:
   * tokens are frame-major, token n = t * S + s with S = N / frames tokens per
     frame (raster order inside a frame);
   * a block is B consecutive tokens of one frame: a frame has

@@ -7,8 +7,7 @@ never calls it, and it shares no code with the CUDA library.
 The page "TurboDiffusion" (section "SageAttention: low-bit quantization")
 says attention is computed at reduced precision, through low-bit
 quantisation, to cut memory traffic and compute while keeping accuracy; it
-gives no format, no scales and no formulas.  Readings taken (listed in
-DESIGN.md):
+gives no format, no scales and no formulas.  Readings taken:
   * Q and K are quantised to FP8 E4M3 (1 sign, 4 exponent bits with bias 7,
     3 mantissa bits; largest finite value 448, smallest subnormal 2^-9, no
     infinities), rounding to nearest with ties to the even mantissa and

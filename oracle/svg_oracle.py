@@ -212,7 +212,7 @@ class RowSelection:
     order: np.ndarray         # all live k-clusters by descending weight (ties: lower id)
     weights: np.ndarray       # normalised weights [Ck]
     undecided: bool           # the cut sits within `band` of p, or between near-equal weights
-    band: float = 0.0         # the band the row was judged with
+    band: float = 0.0         # the band the row was decided with
 
 
 def select_row(weights: np.ndarray, p: float, tol: float,
