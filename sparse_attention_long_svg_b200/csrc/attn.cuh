@@ -1114,61 +1114,88 @@ __global__ void attn_plan_merge_kernel(const int32_t *__restrict__ q_off, const 
 }
 
 // Per (head, q-cluster): number of work items (256 query rows each) and of
-// 128-key tiles per item.  A q-cluster whose block list equals its
-// predecessor's has no items of its own: the first cluster of such a group
-// plans the group's rows (q_end = the group's last row + 1).
-__global__ void attn_plan_count_kernel(const int32_t *__restrict__ q_off,
-                                       const int32_t *__restrict__ k_off,
-                                       const int32_t *__restrict__ sel_count,
-                                       const int32_t *__restrict__ sel_cols, int BH, int Cq, int Ck,
-                                       int max_sel, const int32_t *__restrict__ same_prev,
-                                       int32_t *__restrict__ qtiles, int32_t *__restrict__ ktiles,
-                                       int32_t *__restrict__ q_end) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= BH * Cq) return;
+// 128-key tiles per item; one warp per (head, q-cluster).  A q-cluster whose
+// block list equals its predecessor's has no items of its own: the first
+// cluster of such a group plans the group's rows (q_end = the group's last
+// row + 1).  Selected k-clusters whose row ranges touch (consecutive ids, or
+// ids with only empty clusters between them) form one run, and slots are
+// counted per run, 32 selected clusters at a time with the same ballot rule
+// the attention kernel's item loader merges them by.
+__global__ void __launch_bounds__(256) attn_plan_count_kernel(const int32_t *__restrict__ q_off,
+                                                              const int32_t *__restrict__ k_off,
+                                                              const int32_t *__restrict__ sel_count,
+                                                              const int32_t *__restrict__ sel_cols, int BH, int Cq,
+                                                              int Ck, int max_sel,
+                                                              const int32_t *__restrict__ same_prev,
+                                                              int32_t *__restrict__ qtiles,
+                                                              int32_t *__restrict__ ktiles,
+                                                              int32_t *__restrict__ q_end) {
+  const int lane = threadIdx.x & 31;
+  const int idx = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (idx >= BH * Cq) return;   // warp-uniform
   const int h = idx / Cq, i = idx % Cq;
   if (same_prev[idx]) {   // planned by the first cluster of its group
-    qtiles[idx] = 0;
-    ktiles[idx] = 0;
-    q_end[idx] = 0;
+    if (lane == 0) {
+      qtiles[idx] = 0;
+      ktiles[idx] = 0;
+      q_end[idx] = 0;
+    }
     return;
   }
-  int last = i;
-  while (last + 1 < Cq && same_prev[idx + (last + 1 - i)]) ++last;
-  const int row_end = q_off[h * (Cq + 1) + last + 1];
-  q_end[idx] = row_end;
-  const int nq = row_end - q_off[h * (Cq + 1) + i];
   const int cnt = attn_sel_count(sel_count, idx, max_sel);
   const int32_t *cols = sel_cols + static_cast<size_t>(idx) * Ck;
   const int32_t *ko = k_off + static_cast<size_t>(h) * (Ck + 1);
-  // Selected k-clusters whose row ranges touch (consecutive ids, or ids with
-  // only empty clusters between them) form one run: slots are counted per
-  // run, exactly as the attention kernel's item loader merges them.
-  int slots = 0, run_end = -1, run_len = 0;
-  for (int c = 0; c < cnt; ++c) {
-    const int j = cols[c];
-    if (j < 0 || j >= Ck) {
+  int slots = 0, m = 0, open_x = 0, open_end = -1;   // slots of closed runs; runs opened; the open run
+  for (int c0 = 0; c0 < cnt; c0 += 32) {
+    const int c = c0 + lane;
+    int x = 0, len = 0;
+    if (c < cnt) {
+      const int j = cols[c];
+      if (j >= 0 && j < Ck) {
+        x = ko[j];
+        len = ko[j + 1] - x;
+      } else {
+        record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
+      }
+    }
+    const bool valid = len > 0;
+    const int end = x + len;
+    const unsigned below_mask = (1u << lane) - 1u;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    const unsigned vb = vmask & below_mask;
+    const int pv_end = __shfl_sync(0xffffffffu, end, vb ? 31 - __clz(vb) : 0);
+    const int prev_end = vb ? pv_end : open_end;   // end of the previous non-empty range
+    const bool opens = valid && x != prev_end;
+    const unsigned smask = __ballot_sync(0xffffffffu, opens);
+    const unsigned sb = smask & below_mask;
+    const int ps_x = __shfl_sync(0xffffffffu, x, sb ? 31 - __clz(sb) : 0);
+    int closed = 0;   // slots of the run this lane closes (the run before the one it opens)
+    if (opens && m + __popc(sb) > 0) {
+      const int run_x = sb ? ps_x : open_x;
+      closed = (prev_end - run_x + 7) >> 3;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) closed += __shfl_xor_sync(0xffffffffu, closed, o);
+    slots += closed;
+    if (smask) open_x = __shfl_sync(0xffffffffu, x, 31 - __clz(smask));
+    if (vmask) open_end = __shfl_sync(0xffffffffu, end, 31 - __clz(vmask));
+    m += __popc(smask);
+  }
+  if (m > 0) slots += (open_end - open_x + 7) >> 3;
+  if (lane == 0) {
+    int last = i;
+    while (last + 1 < Cq && same_prev[idx + (last + 1 - i)]) ++last;
+    const int row_end = q_off[h * (Cq + 1) + last + 1];
+    q_end[idx] = row_end;
+    const int nq = row_end - q_off[h * (Cq + 1) + i];
+    int qt = nq > 0 ? (nq + kItemRows - 1) / kItemRows : 0;
+    if (qt > 0 && slots == 0) {
       record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
-      continue;
+      qt = 0;
     }
-    const int r0 = ko[j], len = ko[j + 1] - r0;
-    if (len <= 0) continue;
-    if (r0 == run_end) {
-      run_len += len;
-    } else {
-      slots += (run_len + 7) >> 3;
-      run_len = len;
-    }
-    run_end = r0 + len;
+    qtiles[idx] = qt;
+    ktiles[idx] = (slots + kSlotsPerTile - 1) / kSlotsPerTile;
   }
-  slots += (run_len + 7) >> 3;
-  int qt = nq > 0 ? (nq + kItemRows - 1) / kItemRows : 0;
-  if (qt > 0 && slots == 0) {
-    record_error(SVG_ERR_DEVICE_CHECK, SITE_ATTN_EMPTY_ROW);
-    qt = 0;
-  }
-  qtiles[idx] = qt;
-  ktiles[idx] = (slots + kSlotsPerTile - 1) / kSlotsPerTile;
 }
 
 // Single block: one AttnItem per 256 query rows, in claiming order (a

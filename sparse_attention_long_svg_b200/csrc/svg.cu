@@ -548,7 +548,7 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
   const int max_sel = Ck < AttnCfg<128>::MAX_SEL ? Ck : AttnCfg<128>::MAX_SEL;
   attn_plan_merge_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, sel_count, sel_cols, BH, Cq, Ck, max_sel,
                                                             w.same_prev);
-  attn_plan_count_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
+  attn_plan_count_kernel<<<(pairs + 7) / 8, 256, 0, s>>>(q_off, k_off, sel_count, sel_cols, BH,
                                                             Cq, Ck, max_sel, w.same_prev, w.qtiles, w.ktiles,
                                                             w.q_end);
   attn_plan_emit_kernel<<<1, kAttnBuckets, 0, s>>>(q_off, w.qtiles, w.ktiles, w.q_end, BH, Cq, w.items,
