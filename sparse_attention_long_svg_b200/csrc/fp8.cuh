@@ -8,7 +8,9 @@
 //     all-zero row); K: one float32 scale per head over all its rows, so a key
 //     tile gathered from any rows of the head shares it;
 //   * the stored value is E4M3(x / s), the division in float32.
-// The logits become scale * (q8 . k8) * s_q * s_k; P and V stay bf16.
+// The logits become scale * (q8 . k8) * s_q * s_k; P and V stay bf16.  Rows
+// may be gathered through a permutation on the way (output row i of a head
+// from source row perm[i]), so the permuted bf16 copies are never written.
 #pragma once
 #include <cuda_fp8.h>
 
