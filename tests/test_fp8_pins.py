@@ -85,6 +85,30 @@ def test_fp8_attention_on_representable_inputs_is_exact():
     assert np.allclose(got, want, rtol=0, atol=1e-12) and np.allclose(lse, wlse, atol=1e-12)
 
 
+def test_fp8_attention_with_power_of_two_scales_is_exact():
+    """Rows that are E4M3 values times a power of two (row maximum 448 * 2^e) have scale 2^e
+    exactly, so quantising and dequantising returns them unchanged: the 8-bit attention equals
+    the float64 attention with every scale different from 1 (a dropped or inverted scale fails)."""
+    rng = np.random.default_rng(3)
+    table = np.unique(f8.all_e4m3_values())
+    table = table[np.abs(table) <= 8]
+    N, D = 48, 16
+    eq = rng.integers(-6, 7, N).astype(np.float64)          # per query row
+    q = rng.choice(table, (N, D)); q[:, 0] = 448.0
+    q = q * 2.0 ** eq[:, None]
+    k = rng.choice(table, (N, D)) * 2.0 ** -5; k[3, 2] = 448.0 * 2.0 ** -5   # head scale 2^-5
+    v = rng.standard_normal((N, D))
+    q8, sq = f8.quantize_rows(q)
+    assert np.array_equal(sq, (2.0 ** eq).astype(np.float32)) and np.array_equal(q8 * sq[:, None], q)
+    k8, sk = f8.quantize_tensor(k)
+    assert sk == np.float32(2.0 ** -5) and np.array_equal(k8 * sk, k)
+    q_off = np.array([0, 16, 30, 48]); k_off = np.array([0, 20, 48])
+    sel = [[1], [0, 1], [0]]
+    got, lse = f8.sparse_attention_fp8(q, k, v, q_off, k_off, sel, 0.05)
+    want, wlse = so.sparse_attention(q, k, v, q_off, k_off, sel, 0.05)
+    assert np.allclose(got, want, rtol=0, atol=1e-12) and np.allclose(lse, wlse, rtol=1e-12)
+
+
 def _expect_failure(fn, *args):
     with pytest.raises(AssertionError):
         fn(*args)
@@ -112,3 +136,8 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(f8, "E4M3_MAX", 256.0)
         _expect_failure(test_scales_and_round_trip)
+    # 4. the head's K scale left out of the logits
+    with monkeypatch.context() as m:
+        orig_qt = f8.quantize_tensor
+        m.setattr(f8, "quantize_tensor", lambda x: (orig_qt(x)[0], np.float32(1.0)))
+        _expect_failure(test_fp8_attention_with_power_of_two_scales_is_exact)
