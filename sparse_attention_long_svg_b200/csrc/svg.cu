@@ -62,7 +62,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 // 2-D view [rows, D] of a bf16 (or, with u8, a one-byte-per-channel)
 // tensor; boxes of 128 bytes of channels x box_rows rows, 128-byte swizzle
 // (the tcgen05 K-major / MN-major canonical layout).
-bool make_map_bf16(CUtensorMap *map, const void *base, uint64_t rows, int D, int box_rows, bool u8 = false) {
+bool make_map_2d(CUtensorMap *map, const void *base, uint64_t rows, int D, int box_rows, bool u8 = false) {
   auto enc = encoder();
   if (!enc) return false;
   const int eb = u8 ? 1 : 2;
@@ -365,9 +365,9 @@ svg_status svg_kmeans(const void *x, int BH, int N, int D, int C, int iters, flo
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   const int Cpad = kmeans_cpad(C);
   CUtensorMap mx, mhi, mlo;
-  if (!make_map_bf16(&mx, x, static_cast<uint64_t>(BH) * N, D, 128) ||
-      !make_map_bf16(&mhi, w.hi, static_cast<uint64_t>(BH) * Cpad, D, 128) ||
-      !make_map_bf16(&mlo, w.lo, static_cast<uint64_t>(BH) * Cpad, D, 128))
+  if (!make_map_2d(&mx, x, static_cast<uint64_t>(BH) * N, D, 128) ||
+      !make_map_2d(&mhi, w.hi, static_cast<uint64_t>(BH) * Cpad, D, 128) ||
+      !make_map_2d(&mlo, w.lo, static_cast<uint64_t>(BH) * Cpad, D, 128))
     return SVG_ERR_CUDA;
   kmeans_split_kernel<<<dim3((Cpad + 7) / 8, BH), 256, 0, s>>>(centroids, C, Cpad, D, w.hi, w.lo,
                                                               w.norms, w.num_ties, w.counters);
@@ -559,9 +559,9 @@ svg_status sparse_attn_impl(const void *qp, const void *kp, const void *vp, cons
   AttnMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const uint64_t rows = static_cast<uint64_t>(BH) * N;
-  if (!make_map_bf16(&maps.q, qp, rows, D, 128, fp8)) return SVG_ERR_CUDA;
+  if (!make_map_2d(&maps.q, qp, rows, D, 128, fp8)) return SVG_ERR_CUDA;
   for (int b = 0; b < (gather ? 0 : kNumBoxSizes); ++b)   // gather mode copies rows without tensor maps
-    if (!make_map_bf16(&maps.k[b], kp, rows, D, 8 << b, fp8) || !make_map_bf16(&maps.v[b], vp, rows, D, 8 << b))
+    if (!make_map_2d(&maps.k[b], kp, rows, D, 8 << b, fp8) || !make_map_2d(&maps.v[b], vp, rows, D, 8 << b))
       return SVG_ERR_CUDA;
   AttnParams prm;
   prm.q_off = q_off;
