@@ -233,12 +233,14 @@ def workload_config(wl, n_gpus, heads=None, iters=None, top_p=None):
 
 # ----------------------------------------------------------------------------- GPU leg
 
-def kernel_launches_per_step(iters: int, qk_fp8: bool = False) -> int:
+def kernel_launches_per_step(iters: int, qk_fp8: bool = False, kv_gather: bool = False) -> int:
     """Our kernels per step (counted from the launch sequence in svg.cu)."""
     per_kmeans = 1 + 4 * iters               # split + T x (assign, refine, bucket, accumulate); ||x||^2 in the first assign
     per_permute = 3 + 1                      # hist, scan, scatter + row gather
     if qk_fp8:   # Q's permutation moves no rows; quantise Q per row, K per head (amax, quantise, scale)
         return 2 * per_kmeans + 2 * per_permute - 1 + 1 + 4 + 4
+    if kv_gather:   # K's permutation moves no rows (attention gathers K/V through it)
+        return 2 * per_kmeans + 2 * per_permute - 1 + 1 + 4
     return 2 * per_kmeans + 2 * per_permute + 1 + 4       # select; plan x3 + attention (un-permute fused)
 
 
@@ -579,7 +581,7 @@ def run_svg(args, wl):
                     "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
                     "pipelining": "H2D of step i+1 and D2H of step i-1 overlap the layer of step i "
                                   "(two device buffer sets, three streams)"},
-            "gpu_launches": kernel_launches_per_step(T, bool(args.qk_fp8)) * args.steps,
+            "gpu_launches": kernel_launches_per_step(T, bool(args.qk_fp8), bool(args.kv_gather)) * args.steps,
             "clocks": clocks.summary(),
             "timing": ("CUDA-graph replays of the whole step (stages and per-kernel rooflines from eager steps "
                        "with events; eager %.3f ms per step)" % (eager_ms / args.steps)) if args.graph else

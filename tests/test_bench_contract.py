@@ -24,6 +24,7 @@ def test_launch_count_per_step():
     assert bench.kernel_launches_per_step(5) == 2 * (1 + 4 * 5) + 2 * 4 + 1 + 4 == 55
     assert bench.kernel_launches_per_step(2) == 2 * (1 + 4 * 2) + 13
     assert bench.kernel_launches_per_step(5, qk_fp8=True) == 55 - 1 + 4 == 58
+    assert bench.kernel_launches_per_step(5, kv_gather=True) == 54
 
 
 def test_workload_config_keys():
