@@ -244,6 +244,12 @@ def kernel_launches_per_step(iters: int, qk_fp8: bool = False, kv_gather: bool =
     return 2 * per_kmeans + 2 * per_permute + 1 + 4       # select; plan x3 + attention (un-permute fused)
 
 
+def dynrad_launches_per_step(mode: str) -> int:
+    """Kernels per DynamicRad step: the mask (offsets, [block means,] select) and the attention
+    (plan merge, count, emit + the attention kernel)."""
+    return (3 if mode == "dynamic" else 2) + 4
+
+
 def attention_pairs(layer, wl):
     cnt = layer.sel_count.cpu().numpy()
     cols = layer.sel_cols.cpu().numpy()
@@ -755,7 +761,7 @@ def run_dynrad(args, wl):
                     "d2h_bytes_per_step": int(q.numel() * 2), "ms_per_step": e2e_ms / e2e_steps,
                     "steps": e2e_steps, "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i "
                                                       "(two device buffer sets, three streams)"},
-            "gpu_launches": (6 if mode == "dynamic" else 5) * args.steps,   # mask (offsets, [means,] select) + plan x3 + attention
+            "gpu_launches": dynrad_launches_per_step(mode) * args.steps,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

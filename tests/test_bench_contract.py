@@ -25,6 +25,7 @@ def test_launch_count_per_step():
     assert bench.kernel_launches_per_step(2) == 2 * (1 + 4 * 2) + 13
     assert bench.kernel_launches_per_step(5, qk_fp8=True) == 55 - 1 + 4 == 58
     assert bench.kernel_launches_per_step(5, kv_gather=True) == 54
+    assert bench.dynrad_launches_per_step("static") == 6 and bench.dynrad_launches_per_step("dynamic") == 7
 
 
 def test_workload_config_keys():
